@@ -1,0 +1,158 @@
+"""B200 (sm_100a) fused attention forward: Python binding of the C ABI.
+
+The entry points below have the names and arguments of include/attn_b200.h and
+only marshal arguments: every step of the computation runs in the CUDA kernels
+of libattn_b200.so. There is no CPU fallback; if the library is missing the
+calls raise. `forward`, `quantize_fp8` and `forward_fp8` are torch conveniences
+that allocate outputs with torch (PyTorch serves only for device memory and
+streams) and call the same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
+
+ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(6)
+ATTN_BF16 = 0
+TILE = 128
+
+_lib = None
+
+# (name, restype, argtypes) for every symbol the header declares
+_P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
+    "attn_quantize_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_get_device_status": (_I, [_P]),
+    "attn_status_string": (ctypes.c_char_p, [_I]),
+    "attn_abi_version": (_I, []),
+}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {attn_status_string(status)}")
+
+
+def load():
+    """Load libattn_b200.so (built by exact_attention_forward_11_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run `python -m exact_attention_forward_11_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+# ------------------------------------------------------------------ raw C ABI
+def attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, stream):
+    return load().attn_fwd(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, stream)
+
+
+def attn_quantize_fp8(x, rot, x8, scales, B, H, N, d, stream):
+    return load().attn_quantize_fp8(x, rot, x8, scales, B, H, N, d, stream)
+
+
+def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, scale, causal, stream):
+    return load().attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, scale, causal, stream)
+
+
+def attn_get_device_status(stream):
+    return load().attn_get_device_status(stream)
+
+
+def attn_status_string(status):
+    return load().attn_status_string(int(status)).decode()
+
+
+def attn_abi_version():
+    return load().attn_abi_version()
+
+
+# ------------------------------------------------------------------ torch helpers
+def _stream_ptr(t, stream):
+    import torch
+    s = torch.cuda.current_stream(t.device) if stream is None else stream
+    return s.cuda_stream
+
+
+def _check(status, where):
+    if status != ATTN_OK:
+        raise AttnError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _shape4(q):
+    if q.dim() != 4 or not q.is_contiguous() or not q.is_cuda:
+        raise ValueError("expected a contiguous CUDA tensor [B, H, N, d]")
+    return tuple(q.shape)
+
+
+def forward(q, k, v, causal=False, scale=None, out=None, lse=None, with_lse=True, stream=None):
+    """O, LSE = attention(q, k, v) for bf16 CUDA tensors [B, H, N, d]."""
+    import torch
+    B, H, N, d = _shape4(q)
+    for t in (k, v):
+        if tuple(t.shape) != (B, H, N, d) or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("k, v must match q")
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q must be bf16")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and with_lse:
+        lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    sc = 0.0 if scale is None else float(scale)
+    _check(attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc,
+                    int(bool(causal)), ATTN_BF16, _stream_ptr(q, stream)), "attn_fwd")
+    return out, lse
+
+
+def quantize_fp8(x, rot=None, stream=None):
+    """(codes uint8 [B,H,N,d], scales fp32 [B,H,ceil(N/128)]) of a bf16 tensor."""
+    import torch
+    B, H, N, d = _shape4(x)
+    x8 = torch.empty((B, H, N, d), device=x.device, dtype=torch.uint8)
+    scales = torch.empty((B, H, (N + TILE - 1) // TILE), device=x.device, dtype=torch.float32)
+    _check(attn_quantize_fp8(x.data_ptr(), _ptr(rot), x8.data_ptr(), scales.data_ptr(), B, H, N, d,
+                             _stream_ptr(x, stream)), "attn_quantize_fp8")
+    return x8, scales
+
+
+def forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale=None, out=None, lse=None,
+                with_lse=True, stream=None):
+    """O (bf16), LSE from E4M3 codes and their per-tile scales."""
+    import torch
+    B, H, N, d = _shape4(q8)
+    if out is None:
+        out = torch.empty((B, H, N, d), device=q8.device, dtype=torch.bfloat16)
+    if lse is None and with_lse:
+        lse = torch.empty((B, H, N), device=q8.device, dtype=torch.float32)
+    sc = 0.0 if scale is None else float(scale)
+    _check(attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_scale.data_ptr(), k_scale.data_ptr(),
+                        v_scale.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc, int(bool(causal)),
+                        _stream_ptr(q8, stream)), "attn_fwd_fp8")
+    return out, lse
+
+
+def flops(B, H, N, d, causal):
+    """Algorithmic FLOPs of one forward: 4 B H N^2 d, halved for causal."""
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def default_scale(d):
+    return 1.0 / math.sqrt(d)

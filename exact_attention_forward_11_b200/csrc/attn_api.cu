@@ -1,0 +1,174 @@
+// attn_api.cu - host side of the C ABI declared in include/attn_b200.h.
+//
+// Validates arguments (before anything touches the GPU), encodes TMA tensor maps
+// for the [B*H, N, d] operands, and launches the kernels on the caller's stream.
+// Nothing is allocated per call; the library owns one device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn_b200.h"
+#include "attn_fwd_kernel.cuh"
+#include "fp8_prep_kernel.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+constexpr uint64_t kDefaultWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 3-D map over a contiguous [BH, N, d] tensor: dims {d, N, BH}, box {128 bytes of
+// d, 128 rows, 1}, 128-byte swizzle (the layout the MMA descriptors expect).
+// Rows past N read as zero.
+bool encode_qkv_map(CUtensorMap* map, const void* base, bool fp8, int d, int N, int BH) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  const int elem = fp8 ? 1 : 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem, static_cast<cuuint64_t>(N) * d * elem};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+attn_status check_shape(int B, int H, int N) {
+  if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(B) * H * N;
+  if (rows >= (1ll << 31)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+template <class C>
+attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const float* qs,
+                       const float* ks, const float* vs, int BH, int N, float scale, int causal,
+                       cudaStream_t stream) {
+  CUtensorMap tq, tk, tv;
+  if (!encode_qkv_map(&tq, q, C::FP8, C::D, N, BH) || !encode_qkv_map(&tk, k, C::FP8, C::D, N, BH) ||
+      !encode_qkv_map(&tv, v, C::FP8, C::D, N, BH))
+    return ATTN_ERR_CUDA;
+  auto kern = attn::attn_fwd_sm100<C>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const int QB = (N + attn::kBlockM - 1) / attn::kBlockM;
+  const int npair = (QB + C::Q_TILES - 1) / C::Q_TILES;
+  attn::FwdParams p;
+  p.N = N;
+  p.BH = BH;
+  p.num_units = BH * npair;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.q_scale = qs;
+  p.k_scale = ks;
+  p.v_scale = vs;
+  p.timeout_ns = kDefaultWaitLimitNs;
+  kern<<<p.num_units, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_abi_version(void) { return 1; }
+
+const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    default: return "ATTN_UNKNOWN_STATUS";
+  }
+}
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                     float scale, int causal, int dtype, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
+    return ATTN_ERR_MISALIGNED;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  if (d == 128)
+    return launch_fwd<attn::FwdCfg<128, false>>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+  return launch_fwd<attn::FwdCfg<64, false>>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+}
+
+attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
+                         const float* v_scale, void* o, float* lse, int B, int H, int N, int d, float scale,
+                         int causal, void* stream) {
+  if (q8 == nullptr || k8 == nullptr || v8 == nullptr || o == nullptr || q_scale == nullptr ||
+      k_scale == nullptr || v_scale == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
+    return ATTN_ERR_MISALIGNED;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
+  return launch_fwd<attn::FwdCfg<128, true>>(q8, k8, v8, o, lse, q_scale, k_scale, v_scale, B * H, N, scale, causal,
+                                             static_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* scales, int B, int H, int N, int d,
+                              void* stream) {
+  if (x == nullptr || x8 == nullptr || scales == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (d != attn::kPrepTile) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(x8) || (rot != nullptr && !aligned16(rot))) return ATTN_ERR_MISALIGNED;
+  const int T = (N + attn::kPrepTile - 1) / attn::kPrepTile;
+  if (cudaFuncSetAttribute(attn::fp8_rotate_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           attn::kPrepSmemBytes) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  attn::fp8_rotate_quantize<<<B * H * T, attn::kPrepThreads, attn::kPrepSmemBytes,
+                              static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(rot), static_cast<uint8_t*>(x8),
+      scales, N);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+attn_status attn_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, attn::g_status, sizeof(v)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (v == 0) return ATTN_OK;
+  const uint32_t zero = 0;
+  if (cudaMemcpyToSymbol(attn::g_status, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_ERR_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,123 @@
+/*
+ * attn_b200.h - C ABI of a fused scaled-dot-product attention forward for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation ("Self-Attention, CUDA kernels and FlashAttention", section 1,
+ * eq. Scores and eq. Attention; section 3, tiling / online-softmax / recompute
+ * bullets), computed independently for every (batch b, head h):
+ *
+ *     S   = scale * Q K^T                        (N x N, never stored)
+ *     P   = row-softmax(S), causal: S_ij = -inf for key j > query i
+ *     O   = P V                                  (N x d)
+ *     LSE_i = ln sum_j exp(S_ij)                 (natural log, scale included)
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are dense, contiguous, row-major [B, H, N, d] with d innermost;
+ *     LSE is [B, H, N]; per-tile FP8 scales are [B, H, ceil(N/128)].
+ *   - Every pointer argument is a DEVICE pointer owned by the caller, 16-byte
+ *     aligned. The library never frees or retains caller memory.
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed as
+ *     void*, NULL = the legacy default stream). The host never synchronises.
+ *   - Causal masking is square and top-left aligned: query i sees keys j <= i.
+ *   - scale <= 0 selects the default 1/sqrt(d).
+ *   - Argument errors are detected on the host before anything is launched and
+ *     returned immediately (INVALID_ARG, UNSUPPORTED, MISALIGNED). A failed
+ *     launch returns ATTN_ERR_CUDA. A device-side pipeline wait that exceeds its
+ *     time limit makes the kernel stop early and record ATTN_ERR_TIMEOUT in a
+ *     device status word, read by attn_get_device_status().
+ *   - N >= 1, B >= 1, H >= 1, and B*H*N < 2^31.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad flag        */
+  ATTN_ERR_UNSUPPORTED = 2,  /* head width or dtype this build has no kernel for */
+  ATTN_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned                 */
+  ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed              */
+  ATTN_ERR_TIMEOUT = 5       /* a device pipeline wait ran out (see below)       */
+} attn_status;
+
+typedef enum {
+  ATTN_BF16 = 0              /* bf16 inputs and output, fp32 accumulation        */
+} attn_dtype;
+
+/*
+ * attn_fwd - BF16 attention forward.
+ *   q, k, v : [B, H, N, d] bf16 inputs.
+ *   o       : [B, H, N, d] bf16 output O = softmax(scale Q K^T) V.
+ *   lse     : [B, H, N] fp32 output LSE, or NULL to skip it.
+ *   d       : 64 or 128 (else ATTN_ERR_UNSUPPORTED).
+ *   causal  : 0 or 1.   dtype: ATTN_BF16.
+ * Cites: "Self-Attention, CUDA kernels and FlashAttention", section 1 eq. Attention
+ * (what is computed) and section 3 (tiled, fused, online softmax, only O and the
+ * row statistics written); "FlashAttention scaling, multi-GPU training and weight
+ * quantization", section 1 (FlashAttention-2 loop order and deferred rescaling,
+ * FlashAttention-3 asynchronous copies and warp specialisation).
+ */
+ATTN_API attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                     int B, int H, int N, int d, float scale, int causal, int dtype,
+                     void* stream);
+
+/*
+ * attn_quantize_fp8 - FP8 preparation of one tensor (incoherent processing and
+ * block quantisation, "FlashAttention scaling, multi-GPU training and weight
+ * quantization", section 1, FlashAttention-3 FP8 bullet).
+ *   x      : [B, H, N, d] bf16 input.
+ *   rot    : [d, d] bf16 orthogonal matrix (row-major), or NULL for no rotation
+ *            (V is quantised without rotation).
+ *   x8     : [B, H, N, d] output E4M3 codes (one byte each).
+ *   scales : [B, H, ceil(N/128)] fp32 output, one per tile of 128 tokens x d.
+ *   d      : 128 (else ATTN_ERR_UNSUPPORTED).
+ * Definition: y = x rot accumulated in fp32 in increasing k order;
+ * scale = max|y| over the tile / 448 (1 for an all-zero tile);
+ * code = E4M3 round-to-nearest-even, saturating, of y / scale.
+ */
+ATTN_API attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* scales,
+                              int B, int H, int N, int d, void* stream);
+
+/*
+ * attn_fwd_fp8 - attention forward on block-quantised E4M3 inputs.
+ *   q8, k8, v8 : [B, H, N, d] E4M3 codes (q8, k8 rotated by the same orthogonal
+ *                matrix, which leaves Q K^T unchanged).
+ *   q_scale, k_scale, v_scale : [B, H, ceil(N/128)] fp32 tile scales; the
+ *                value of a code is decode(code) * scale of its 128-token tile.
+ *   o   : [B, H, N, d] bf16 output.  lse: [B, H, N] fp32 or NULL.
+ *   d   : 128 (else ATTN_ERR_UNSUPPORTED).
+ * Computes the attention of the dequantised values; P is re-quantised to E4M3
+ * on chip for the P V product (the error this adds is within the FP8 tolerance).
+ */
+ATTN_API attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
+                         const float* q_scale, const float* k_scale, const float* v_scale,
+                         void* o, float* lse, int B, int H, int N, int d, float scale,
+                         int causal, void* stream);
+
+/*
+ * attn_get_device_status - synchronises `stream`, then reads and clears the
+ * device status word that kernels set when a pipeline wait timed out.
+ * Returns ATTN_OK, ATTN_ERR_TIMEOUT, or ATTN_ERR_CUDA if the read failed.
+ */
+ATTN_API attn_status attn_get_device_status(void* stream);
+
+/* attn_status_string - static, human-readable name of a status code. */
+ATTN_API const char* attn_status_string(int status);
+
+/* attn_abi_version - version of this ABI (incremented on incompatible change). */
+ATTN_API int attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_H */

@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports every symbol include/attn_b200.h declares, and
+rejects bad arguments on the host before any CUDA call (so this runs without a GPU)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_b200.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_attention_forward_11_b200 import build
+    build.build()
+    import exact_attention_forward_11_b200 as m
+    return m
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    assert {"attn_fwd", "attn_fwd_fp8", "attn_quantize_fp8", "attn_get_device_status",
+            "attn_status_string", "attn_abi_version"} <= set(syms)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = lib.LIB_PATH
+    out = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for s in declared_symbols():
+        assert s in exported, s
+    handle = ctypes.CDLL(so)
+    for s in declared_symbols():
+        assert getattr(handle, s) is not None
+    # the binding wraps every declared symbol under the same name
+    for s in declared_symbols():
+        assert s in lib.SIGNATURES and callable(getattr(lib, s))
+
+
+def test_status_strings_and_version(lib):
+    assert lib.attn_abi_version() == 1
+    assert lib.attn_status_string(0) == "ATTN_OK"
+    assert lib.attn_status_string(5) == "ATTN_ERR_TIMEOUT"
+    assert lib.attn_status_string(99) == "ATTN_UNKNOWN_STATUS"
+
+
+FAKE = 0x100000  # 16-byte aligned, never dereferenced: validation fails first
+
+
+def test_fwd_argument_validation(lib):
+    f = lib.attn_fwd
+    ok = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, H=1, N=8, d=64, scale=0.0, causal=0, dtype=0,
+              stream=None)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["N"], a["d"], a["scale"],
+                 a["causal"], a["dtype"], a["stream"])
+    assert call(q=None) == lib.ATTN_ERR_INVALID_ARG
+    assert call(o=None) == lib.ATTN_ERR_INVALID_ARG
+    assert call(N=0) == lib.ATTN_ERR_INVALID_ARG
+    assert call(B=-1) == lib.ATTN_ERR_INVALID_ARG
+    assert call(causal=2) == lib.ATTN_ERR_INVALID_ARG
+    assert call(scale=float("nan")) == lib.ATTN_ERR_INVALID_ARG
+    assert call(B=1 << 16, H=1 << 10, N=1 << 10) == lib.ATTN_ERR_INVALID_ARG  # rows overflow int32
+    assert call(d=96) == lib.ATTN_ERR_UNSUPPORTED
+    assert call(d=256) == lib.ATTN_ERR_UNSUPPORTED
+    assert call(dtype=1) == lib.ATTN_ERR_UNSUPPORTED
+    assert call(k=FAKE + 2) == lib.ATTN_ERR_MISALIGNED
+    assert call(lse=FAKE + 4) == lib.ATTN_ERR_MISALIGNED
+
+
+def test_fp8_argument_validation(lib):
+    f = lib.attn_fwd_fp8
+    base = [FAKE] * 7 + [None, 1, 1, 8, 128, 0.0, 0, None]
+    assert f(*base[:3], None, *base[4:]) == lib.ATTN_ERR_INVALID_ARG
+    args = list(base)
+    args[11] = 64
+    assert f(*args) == lib.ATTN_ERR_UNSUPPORTED
+    args = list(base)
+    args[2] = FAKE + 1
+    assert f(*args) == lib.ATTN_ERR_MISALIGNED
+    q = lib.attn_quantize_fp8
+    assert q(None, None, FAKE, FAKE, 1, 1, 8, 128, None) == lib.ATTN_ERR_INVALID_ARG
+    assert q(FAKE, None, FAKE, FAKE, 1, 1, 8, 64, None) == lib.ATTN_ERR_UNSUPPORTED
+    assert q(FAKE, FAKE + 8, FAKE, FAKE, 1, 1, 8, 128, None) == lib.ATTN_ERR_MISALIGNED
+
+
+def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
+    import exact_attention_forward_11_b200 as m
+    monkeypatch.setattr(m, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(m, "_lib", None)
+    with pytest.raises(RuntimeError, match="not built"):
+        m.load()
