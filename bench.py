@@ -1,0 +1,432 @@
+"""Benchmark of the fused attention forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one full pass of the hot path (one attn_fwd launch, or for the FP8
+workload the three preparation launches plus attn_fwd_fp8) over one batch of
+synthetic inputs already resident in HBM. The default workload is the LLM
+training shape B=4, H=32, N=4096, d=128, causal, bf16: its inputs (403 MB) are
+larger than L2 (126 MB), so no L2 flush is needed between timed iterations.
+Timing uses CUDA events on the launching stream, W warm-up steps, then exactly K
+timed steps bracketed by a barrier and device synchronisation; for N > 1 each
+rank runs its own replica of the workload (the (batch, head) units are fully
+independent, so the job shards with no data-path collective: weak scaling) and
+the time is the maximum over ranks.
+
+`--impl reference` times the fp64 CPU oracle (the only other implementation that
+exists for this path) on a bounded sample of the same workload, on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+import workloads  # noqa: E402
+
+METRIC = "attention fwd TFLOPS (BF16 / FP8) and % of B200 tensor-core peak"
+DEFAULT_WORKLOAD = "llm_train_causal"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch size (small profiling captures only)")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(backend, world):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value, world, device=None):
+    """Maximum of a float over all ranks (plumbing for the timing contract)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def shard_seed(w, rank):
+    """Each rank draws its own replica of the workload (different data, same shape)."""
+    return w.seed + 7919 * rank
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons with nvidia-smi while running."""
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu_id), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.15)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.1)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        import statistics
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                sms.append(float(parts[0]))
+                maxs.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def gpu_smi_id(dev, local):
+    """nvidia-smi identifier (UUID) of a torch device, falling back to its index."""
+    import torch
+    uid = str(getattr(torch.cuda.get_device_properties(dev), "uuid", "") or "")
+    if uid:
+        return uid if uid.startswith("GPU-") else "GPU-" + uid
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    return vis.split(",")[local] if vis else str(local)
+
+
+def measured_peaks():
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d.get("bf16_tflops"), d.get("hbm_gbs"), "measured"
+    return 1590.0, 6650.0, "fallback"
+
+
+# ------------------------------------------------------------------ our arm
+class Step:
+    """One pass of the hot path over resident inputs; returns launches per step."""
+
+    def __init__(self, lib, w, x, dev):
+        import torch
+        self.lib, self.w = lib, w
+        self.dev = dev
+        self.q, self.k, self.v = (x[n].to(dev) for n in ("q", "k", "v"))
+        self.o = torch.empty((w.B, w.H, w.N, w.d), device=dev, dtype=torch.bfloat16)
+        self.lse = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
+        if w.fp8:
+            self.rot = x["rot"].to(dev)
+            T = (w.N + 127) // 128
+            self.codes = [torch.empty((w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8) for _ in range(3)]
+            self.scales = [torch.empty((w.B, w.H, T), device=dev, dtype=torch.float32) for _ in range(3)]
+        self.launches = 4 if w.fp8 else 1
+
+    def run_device(self, stream):
+        lib, w = self.lib, self.w
+        s = stream.cuda_stream
+        if not w.fp8:
+            st = lib.attn_fwd(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(), self.o.data_ptr(),
+                              self.lse.data_ptr(), w.B, w.H, w.N, w.d, w.scale, int(w.causal), lib.ATTN_BF16, s)
+            if st:
+                raise lib.AttnError(st, "attn_fwd")
+            return
+        for src, rot, c8, sc in zip((self.q, self.k, self.v), (self.rot, self.rot, None), self.codes, self.scales):
+            st = lib.attn_quantize_fp8(src.data_ptr(), None if rot is None else rot.data_ptr(), c8.data_ptr(),
+                                       sc.data_ptr(), w.B, w.H, w.N, w.d, s)
+            if st:
+                raise lib.AttnError(st, "attn_quantize_fp8")
+        st = lib.attn_fwd_fp8(*(c.data_ptr() for c in self.codes), *(c.data_ptr() for c in self.scales),
+                              self.o.data_ptr(), self.lse.data_ptr(), w.B, w.H, w.N, w.d, w.scale,
+                              int(w.causal), s)
+        if st:
+            raise lib.AttnError(st, "attn_fwd_fp8")
+
+
+def time_device(step, stream, steps, warmup, world, dev):
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(warmup):
+            step.run_device(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step.run_device(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world, dev)
+    return e0.elapsed_time(e1)  # ms for `steps` steps, this rank
+
+
+def time_e2e(lib, w, x, dev, stream, steps):
+    """Same metric end to end through the public Python API: pinned host inputs
+    copied in, forward, O and LSE read back, every step inside the timed region."""
+    import torch
+    host = {n: x[n].pin_memory() for n in ("q", "k", "v")}
+    o_host = torch.empty((w.B, w.H, w.N, w.d), dtype=torch.bfloat16).pin_memory()
+    l_host = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+    dq, dk, dv = (torch.empty_like(host[n], device=dev) for n in ("q", "k", "v"))
+    do = torch.empty((w.B, w.H, w.N, w.d), device=dev, dtype=torch.bfloat16)
+    dl = torch.empty((w.B, w.H, w.N), device=dev, dtype=torch.float32)
+    extra = {}
+    if w.fp8:
+        extra["rot"] = x["rot"].to(dev)
+
+    def one():
+        with torch.cuda.stream(stream):
+            dq.copy_(host["q"], non_blocking=True)
+            dk.copy_(host["k"], non_blocking=True)
+            dv.copy_(host["v"], non_blocking=True)
+            if w.fp8:
+                q8, qs = lib.quantize_fp8(dq, extra["rot"], stream=stream)
+                k8, ks = lib.quantize_fp8(dk, extra["rot"], stream=stream)
+                v8, vs = lib.quantize_fp8(dv, None, stream=stream)
+                lib.forward_fp8(q8, k8, v8, qs, ks, vs, causal=w.causal, out=do, lse=dl, stream=stream)
+            else:
+                lib.forward(dq, dk, dv, causal=w.causal, out=do, lse=dl, stream=stream)
+            o_host.copy_(do, non_blocking=True)
+            l_host.copy_(dl, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v"))
+    d2h = o_host.numel() * 2 + l_host.numel() * 4
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    init_dist("nccl", world)
+    import exact_attention_forward_11_b200 as lib
+    lib.load()
+    w = workloads.WORKLOADS[args.workload]
+    if args.batch is not None:
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch)
+    x = workloads.make_qkv(w.B, w.H, w.N, w.d, shard_seed(w, rank), w.outliers)
+    x = {"q": x[0], "k": x[1], "v": x[2]}
+    if w.fp8:
+        x["rot64"], x["rot"] = workloads.make_rotation(w.d, w.seed + 7919)
+    stream = torch.cuda.Stream(dev)
+    step = Step(lib, w, x, dev)
+    with ClockSampler(gpu_smi_id(dev, local)) as clk:
+        ms_rank = time_device(step, stream, args.steps, max(3, args.warmup), world, dev)
+    st = lib.attn_get_device_status(stream.cuda_stream)
+    if st != lib.ATTN_OK:
+        raise lib.AttnError(st, "device status")
+    ms_total = max_over_ranks(ms_rank, world, dev)
+    ms_step = ms_total / args.steps
+    flops_rank = w.flops
+    tflops = flops_rank * world / (ms_step * 1e-3) / 1e12
+    # e2e through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e_ms, h2d, d2h = time_e2e(lib, w, x, dev, stream, args.e2e_steps)
+        e2e_ms = max_over_ranks(e2e_ms, world, dev)
+        e2e = {"value": round(flops_rank * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
+    peak, hbm, peak_src = measured_peaks()
+    if w.fp8:
+        peak = peak * 2  # FP8 dense = 2x BF16 (nominal ratio)
+    # the dominant kernel is the attention kernel (one launch per BF16 step)
+    kernel_ms = ms_rank / args.steps
+    achieved = flops_rank / (kernel_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(args.workload),
+            "peak_source": f"{peak_src} bf16 burst" + (" x2 (fp8 nominal ratio)" if w.fp8 else ""),
+            "kernel": "attn_fwd_sm100" + ("+fp8_rotate_quantize" if w.fp8 else "")}
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline(w, budget_s=float(os.environ.get("ATTN_CPU_BASELINE_S", "15")))
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": round(tflops, 3), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if w.fp8 else "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B * world, "B_per_gpu": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "flops_per_step_per_gpu": w.flops,
+                   "parallelism": f"replicas x{world} (independent (b,h) units, no collective)",
+                   "l2": "inputs larger than L2 (no flush)" if 3 * w.B * w.H * w.N * w.d * 2 > L2_BYTES
+                   else "inputs smaller than L2"},
+        "pct_of_peak": round(100 * tflops / world / peak, 2),
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": step.launches * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def traffic_per_launch(workload):
+    """DRAM bytes per launch from the committed ncu summary, if one matches."""
+    path = os.path.join(HERE, "profiles", "traffic.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f).get(workload)
+    return None
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def oracle_sample(w, rows_per_head, heads, seed):
+    """A bounded sample of the workload for the fp64 oracle: `heads` heads and
+    `rows_per_head` query rows each. Returns (callable, algorithmic FLOPs)."""
+    import numpy as np
+    import torch
+    gen = torch.Generator().manual_seed(seed)
+    H = heads
+    q = torch.randn((H, w.N, w.d), generator=gen).to(torch.bfloat16).double().numpy()
+    k = torch.randn((H, w.N, w.d), generator=gen).to(torch.bfloat16).double().numpy()
+    v = torch.randn((H, w.N, w.d), generator=gen).to(torch.bfloat16).double().numpy()
+    rows = sorted(set(torch.randint(0, w.N, (rows_per_head,), generator=gen).tolist()))
+    if w.causal:
+        fl = sum(4.0 * (i + 1) * w.d for i in rows) * H
+    else:
+        fl = 4.0 * w.N * w.d * len(rows) * H
+    from oracle import attention_fp64
+
+    def call():
+        return attention_fp64(q, k, v, w.scale, w.causal, rows=rows)
+    return call, fl, f"{H} head(s) x {len(rows)} query rows of {w.name} (N={w.N}, d={w.d})"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, budget_s=15.0):
+    """Times the oracle as it stands on the host cores, on a bounded sample."""
+    rows = 256
+    call, fl, desc = oracle_sample(w, rows, 1, 12345)
+    t0 = time.perf_counter()
+    call()
+    one = time.perf_counter() - t0
+    reps = max(1, int(budget_s / max(one, 1e-3)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        call()
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": desc + f", fp64 numpy, {reps} repetitions"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS[args.workload]
+    # each step: one head x 64 query rows of the workload (bounded so that
+    # warm-up + K steps finish within minutes)
+    call, fl, desc = oracle_sample(w, 64, 1, 4321)
+    for _ in range(max(1, args.warmup)):
+        call()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        call()
+    dt = (time.perf_counter() - t0) / args.steps
+    v = fl / dt / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal},
+            "cpu_baseline": {"value": round(v, 6), "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
+                             "sample": desc + " per step"},
+            "e2e": {"value": round(v, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -67,7 +67,11 @@ struct FwdCfg {
   static constexpr int UMMA_K = FP8 ? 32 : 16;                  // K elements per MMA
   static constexpr int S_KSTEPS = D / UMMA_K;
   static constexpr int PV_KSTEPS = kBlockN / UMMA_K;
-  static constexpr int P_COLS = kBlockN * ELEM / 4;             // TMEM columns holding P
+  // P in TMEM: bf16 pairs (64 columns), or for FP8 two E4M3 terms hi + lo of
+  // each value (32 + 32 columns), so the P V product sees ~7 significant bits
+  // of P instead of E4M3's 4; P V then runs over K = 256 (hi | lo) x (V ; V).
+  static constexpr int P_COLS = 64;
+  static constexpr int PV_KSTEPS_TOTAL = FP8 ? 2 * PV_KSTEPS : PV_KSTEPS;
   static constexpr int NUM_SOFTMAX_THREADS = 128 * Q_TILES;
   static constexpr int PRODUCER_WARP = NUM_SOFTMAX_THREADS / 32;
   static constexpr int MMA_WARP = PRODUCER_WARP + 1;
@@ -244,8 +248,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // O_t (+)= P_t V_j: P from TMEM (over S_t), V MN-major in shared memory
       auto issue_pv = [&](int t, uint32_t v_addr, bool acc) {
 #pragma unroll
-        for (int kk = 0; kk < C::PV_KSTEPS; ++kk) {
-          const uint64_t db = smem_desc(v_addr + kk * C::UMMA_K * 128, C::CHUNK_BYTES, 1024);
+        for (int kk = 0; kk < C::PV_KSTEPS_TOTAL; ++kk) {
+          const uint64_t db = smem_desc(v_addr + (kk % C::PV_KSTEPS) * C::UMMA_K * 128, C::CHUNK_BYTES, 1024);
           const uint32_t a_tmem = tmem_base + t * 128 + kk * 8;
           if constexpr (C::FP8)
             mma_f8_ts(tmem_base + C::O_COL0 + t * C::D, a_tmem, db, idesc_o, (acc || kk > 0) ? 1u : 0u);
@@ -373,6 +377,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           pk[i] = pack_bf16x2(p0, p1);
         }
       } else {
+        // P = hi + lo, both E4M3: hi = e4m3(p), lo = e4m3(p - hi) (residual in f16)
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(sr[4 * i]), c, -m_exp));
@@ -380,7 +385,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const float p2 = ex2_approx(fmaf(__uint_as_float(sr[4 * i + 2]), c, -m_exp));
           const float p3 = ex2_approx(fmaf(__uint_as_float(sr[4 * i + 3]), c, -m_exp));
           sum += (p0 + p1) + (p2 + p3);
-          pk[i] = pack_e4m3x4(p0, p1, p2, p3);
+          const uint32_t h01 = pack_f16x2(p0, p1), h23 = pack_f16x2(p2, p3);
+          const uint16_t hi01 = e4m3x2_from_f16x2(h01), hi23 = e4m3x2_from_f16x2(h23);
+          const uint16_t lo01 = e4m3x2_from_f16x2(hsub2_u32(h01, f16x2_from_e4m3x2(hi01)));
+          const uint16_t lo23 = e4m3x2_from_f16x2(hsub2_u32(h23, f16x2_from_e4m3x2(hi23)));
+          pk[i] = static_cast<uint32_t>(hi01) | (static_cast<uint32_t>(hi23) << 16);
+          pk[32 + i] = static_cast<uint32_t>(lo01) | (static_cast<uint32_t>(lo23) << 16);
         }
         // back to the units of 2^m_use
         sum *= ex2_approx(-v_log2_ratio - C::P_PRESCALE_LOG2);
@@ -399,12 +409,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         }
       }
       // P_t over the first columns of S_t
-      if constexpr (C::P_COLS == 64) {
-        tmem_st32(s_tm + 0, pk);
-        tmem_st32(s_tm + 32, pk + 32);
-      } else {
-        tmem_st32(s_tm + 0, pk);
-      }
+      tmem_st32(s_tm + 0, pk);
+      tmem_st32(s_tm + 32, pk + 32);
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(p_full + t);
