@@ -33,7 +33,9 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-constexpr uint64_t kDefaultWaitLimitNs = 1000000000ull;  // 1 s per pipeline wait
+// Each pipeline wait gives up after 2^31 SM cycles: about 1.1 s at the 1965 MHz
+// maximum clock, longer at lower clocks.
+constexpr uint64_t kWaitLimitCycles = 1ull << 31;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -86,7 +88,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.q_scale = qs;
   p.k_scale = ks;
   p.v_scale = vs;
-  p.timeout_ns = kDefaultWaitLimitNs;
+  p.timeout_cycles = kWaitLimitCycles;
   kern<<<p.num_units, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

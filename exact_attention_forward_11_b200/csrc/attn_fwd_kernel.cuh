@@ -15,11 +15,13 @@
 // Blackwell: accumulators live in tensor memory (TMEM), the MMAs are tcgen05
 // issued by one thread, and P goes back into TMEM as the A operand of P V.
 //
-// CTA layout (Q_TILES = 2): 10 warps.
+// CTA layout (Q_TILES = 2): 12 warps = 3 warpgroups.
 //   warps 0-3  softmax group for Q tile 0 (one thread per query row)
 //   warps 4-7  softmax group for Q tile 1
 //   warp  8    TMA producer (one elected lane)
 //   warp  9    MMA issuer (one elected lane); owns the TMEM allocation
+//   warps 10-11 idle (they complete the control warpgroup, whose registers are
+//              handed to the softmax warpgroups)
 // TMEM (512 columns x 128 lanes of 32 bit):
 //   S_t  columns [128 t, 128 t + 128)   fp32 scores of tile t; P_t (bf16 pairs or
 //                                        E4M3 quads) is written over its first
@@ -72,10 +74,19 @@ struct FwdCfg {
   // of P instead of E4M3's 4; P V then runs over K = 256 (hi | lo) x (V ; V).
   static constexpr int P_COLS = 64;
   static constexpr int PV_KSTEPS_TOTAL = FP8 ? 2 * PV_KSTEPS : PV_KSTEPS;
+  // P is handed to the MMA in P_CHUNKS chunks of 64 keys, each with its own
+  // barrier, so P V of a tile starts under the tile's remaining exponentials.
+  static constexpr int P_CHUNKS = 2;
+  static constexpr int KEYS_PER_CHUNK = kBlockN / P_CHUNKS;
   static constexpr int NUM_SOFTMAX_THREADS = 128 * Q_TILES;
   static constexpr int PRODUCER_WARP = NUM_SOFTMAX_THREADS / 32;
   static constexpr int MMA_WARP = PRODUCER_WARP + 1;
-  static constexpr int THREADS = NUM_SOFTMAX_THREADS + 64;
+  static constexpr int THREADS = NUM_SOFTMAX_THREADS + 128;   // + one control warpgroup
+  // Register split (launch: 65536 / 384 -> 168 per thread = 64512 in total):
+  // softmax warpgroups 216, control warpgroup 64: 2*128*216 + 128*64 = 63488.
+  static constexpr uint32_t REGS_SOFTMAX = 216;
+  static constexpr uint32_t REGS_CONTROL = 64;
+  static_assert(Q_TILES * 128 * REGS_SOFTMAX + 128 * REGS_CONTROL <= 168 * THREADS, "register split");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t O_COL0 = 256;
   // Lazy rescaling: the running maximum is only moved when a new block raises it
@@ -83,12 +94,23 @@ struct FwdCfg {
   // FP8 P must stay below 448 after a 2^8 pre-scale, so it moves every time.
   static constexpr float RESCALE_THRESHOLD = FP8 ? 0.0f : 8.0f;
   static constexpr float P_PRESCALE_LOG2 = 8.0f;  // FP8 only
+  // Pairs of P values (by index mod 8) whose exp2 runs as a polynomial on the
+  // FMA pipe instead of the MUFU unit, in blocks that need no masking. MUFU
+  // throughput alone (16/clk/SM) matches the tensor cores at d = 128, so part
+  // of the exponentials moves to the otherwise idler FMA pipe.
+#ifndef ATTN_POLY_MASK_BF16
+#define ATTN_POLY_MASK_BF16 0x00u
+#endif
+#ifndef ATTN_POLY_MASK_FP8
+#define ATTN_POLY_MASK_FP8 0x22u
+#endif
+  static constexpr uint32_t POLY_MASK = FP8 ? ATTN_POLY_MASK_FP8 : ATTN_POLY_MASK_BF16;
 
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_KV = SMEM_Q + Q_TILES * TILE_BYTES;
   static constexpr int SMEM_BAR = SMEM_KV + NSLOT * TILE_BYTES;
-  static constexpr int NUM_BARS = 1 + 2 * NSLOT + 3 * Q_TILES + 1;
+  static constexpr int NUM_BARS = 1 + 2 * NSLOT + (2 + P_CHUNKS) * Q_TILES + 1;
   static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
 };
@@ -104,20 +126,173 @@ struct FwdParams {
   const float* q_scale;   // FP8: [BH, ceil(N/128)]
   const float* k_scale;
   const float* v_scale;
-  uint64_t timeout_ns;
+  uint64_t timeout_cycles;  // per pipeline wait, in SM cycles
 };
 
 // Bounded wait that ignores the abort word (used only while draining after an
 // abort, so that in-flight copies and MMAs land before the CTA exits).
-__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  const uint64_t t0 = b200::global_timer_ns();
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_cycles) {
+  const uint64_t t0 = b200::sm_clock();
   while (!b200::mbar_try_wait(bar, parity)) {
-    if (b200::global_timer_ns() - t0 > limit_ns) return false;
+    if (b200::sm_clock() - t0 > limit_cycles) return false;
   }
   return true;
 }
 
 __device__ __forceinline__ void record_timeout() { atomicOr(&g_status, kStatusTimeout); }
+
+// 2^x for a pair of fp32 arguments on the FMA/ALU pipes. Cody-Waite style
+// reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low
+// mantissa bits), f in [-1/2, 1/2]; 2^f from a degree-3 polynomial minimising the
+// relative error (Remez exchange, fit_exp2_poly.py: max relative error 7.5e-5);
+// 2^n is applied by adding n to the exponent field. Arguments are clamped at
+// -125 so the result stays normal; 2^-125 stands in for 0, far below any P value
+// that survives bf16 / E4M3 rounding next to the row maximum (P <= 2^8).
+constexpr float kExp2C0 = 0.9999280571937561f;
+constexpr float kExp2C1 = 0.6932609677314758f;
+constexpr float kExp2C2 = 0.2426111251115799f;
+constexpr float kExp2C3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
+
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& p0, float& p1) {
+  using namespace b200;
+  const uint64_t xc = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t tt = f2_add(xc, f2_pack(kRoundMagic, kRoundMagic));   // n in the low mantissa bits
+  const uint64_t n = f2_add(tt, f2_pack(-kRoundMagic, -kRoundMagic));  // round(x), exact
+  float f0, f1, t0, t1;
+  f2_unpack(f2_sub(xc, n), f0, f1);                                    // f = x - n in [-1/2, 1/2]
+  f2_unpack(tt, t0, t1);
+  // Horner with scalar FMAs (the packed FMA would compete with MUFU for issue)
+  float q0 = fmaf(f0, kExp2C3, kExp2C2), q1 = fmaf(f1, kExp2C3, kExp2C2);
+  q0 = fmaf(q0, f0, kExp2C1);
+  q1 = fmaf(q1, f1, kExp2C1);
+  q0 = fmaf(q0, f0, kExp2C0);
+  q1 = fmaf(q1, f1, kExp2C0);
+  p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
+template <uint32_t POLY_MASK>
+__device__ __forceinline__ void exp2_pair(float x0, float x1, int i, float& p0, float& p1) {
+  if ((POLY_MASK >> (i & 7)) & 1u) {
+    exp2_poly_x2(x0, x1, p0, p1);
+  } else {
+    p0 = b200::ex2_approx(x0);
+    p1 = b200::ex2_approx(x1);
+  }
+}
+
+// Maximum of 128 values with 3-input max in eight independent chains.
+__device__ __forceinline__ float row_max128(const uint32_t (&sr)[128]) {
+  using b200::max3f;
+  float a[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float m = max3f(__uint_as_float(sr[16 * k]), __uint_as_float(sr[16 * k + 1]), __uint_as_float(sr[16 * k + 2]));
+#pragma unroll
+    for (int j = 3; j < 15; j += 2)
+      m = max3f(m, __uint_as_float(sr[16 * k + j]), __uint_as_float(sr[16 * k + j + 1]));
+    a[k] = fmaxf(m, __uint_as_float(sr[16 * k + 15]));
+  }
+  return max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
+}
+
+// P = 2^(s c - m) for keys [32 ch, 32 ch + 32) of one row, as 16 bf16 pairs in
+// pk; adds the fp32 values to the packed accumulators. The scale-and-subtract
+// is a scalar FMA per element (a packed FMA would compete with MUFU for issue);
+// the sums use packed adds, which do not.
+template <uint32_t POLY_MASK, int PAIRS = 16>
+__device__ __forceinline__ void p_chunk_bf16(const uint32_t (&sr)[128], int ch, float c, float m,
+                                             uint64_t (&acc)[4], uint32_t (&pk)[PAIRS]) {
+  using namespace b200;
+#pragma unroll
+  for (int i = 0; i < PAIRS; ++i) {
+    const int k = 2 * PAIRS * ch + 2 * i;
+    float p0, p1;
+    exp2_pair<POLY_MASK>(fmaf(__uint_as_float(sr[k]), c, -m), fmaf(__uint_as_float(sr[k + 1]), c, -m), i, p0, p1);
+    acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+    pk[i] = pack_bf16x2(p0, p1);
+  }
+}
+
+// FP8 variant: P = hi + lo with hi = e4m3(p), lo = e4m3(p - hi) (residual in
+// f16); the chunk's 32 keys give 8 hi words and 8 lo words (four codes each).
+template <uint32_t POLY_MASK, int QUADS = 8>
+__device__ __forceinline__ void p_chunk_fp8(const uint32_t (&sr)[128], int ch, float c, float m,
+                                            uint64_t (&acc)[4], uint32_t (&hi)[QUADS], uint32_t (&lo)[QUADS]) {
+  using namespace b200;
+#pragma unroll
+  for (int i = 0; i < QUADS; ++i) {
+    const int k = 4 * QUADS * ch + 4 * i;
+    float p0, p1, p2, p3;
+    exp2_pair<POLY_MASK>(fmaf(__uint_as_float(sr[k]), c, -m), fmaf(__uint_as_float(sr[k + 1]), c, -m), 2 * i, p0,
+                         p1);
+    exp2_pair<POLY_MASK>(fmaf(__uint_as_float(sr[k + 2]), c, -m), fmaf(__uint_as_float(sr[k + 3]), c, -m), 2 * i + 1,
+                         p2, p3);
+    acc[(2 * i) & 3] = f2_add(acc[(2 * i) & 3], f2_pack(p0, p1));
+    acc[(2 * i + 1) & 3] = f2_add(acc[(2 * i + 1) & 3], f2_pack(p2, p3));
+    const uint32_t h01 = pack_f16x2(p0, p1), h23 = pack_f16x2(p2, p3);
+    const uint16_t hi01 = e4m3x2_from_f16x2(h01), hi23 = e4m3x2_from_f16x2(h23);
+    const uint16_t lo01 = e4m3x2_from_f16x2(hsub2_u32(h01, f16x2_from_e4m3x2(hi01)));
+    const uint16_t lo23 = e4m3x2_from_f16x2(hsub2_u32(h23, f16x2_from_e4m3x2(hi23)));
+    hi[i] = static_cast<uint32_t>(hi01) | (static_cast<uint32_t>(hi23) << 16);
+    lo[i] = static_cast<uint32_t>(lo01) | (static_cast<uint32_t>(lo23) << 16);
+  }
+}
+
+// Hands a P chunk to the MMA thread: each thread waits for its own TMEM stores
+// and arrives (the barrier counts the 128 threads of the group).
+__device__ __forceinline__ void release_chunk(uint64_t* bar) {
+  b200::tmem_st_wait();
+  b200::tc_fence_before();
+  b200::mbar_arrive(bar);
+}
+
+// Writes P chunk by chunk into TMEM (over the first columns of S_t) and
+// releases each chunk to the MMA thread; returns the fp32 row sum. Software
+// pipelined: chunk c is stored, chunk c+1 is computed, and only then does the
+// thread wait for chunk c's store and release it, so the store latency hides
+// under the next chunk's exponentials.
+template <class C, uint32_t POLY_MASK>
+__device__ __forceinline__ float p_row_to_tmem(const uint32_t (&sr)[128], float c, float m, uint32_t s_tm,
+                                               uint64_t* p_full_t) {
+  using namespace b200;
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+  constexpr int COLS = 64 / C::P_CHUNKS;   // TMEM columns of P per chunk (bf16 pairs / hi+lo quads)
+#pragma unroll
+  for (int ch = 0; ch < C::P_CHUNKS; ++ch) {
+    if constexpr (!C::FP8) {
+      uint32_t pk[COLS];
+      p_chunk_bf16<POLY_MASK, COLS>(sr, ch, c, m, acc, pk);
+      if (ch > 0) {
+        release_chunk(p_full_t + ch - 1);
+      }
+      if constexpr (COLS == 16) tmem_st16(s_tm + COLS * ch, pk);
+      else if constexpr (COLS == 32) tmem_st32(s_tm + COLS * ch, pk);
+      else { tmem_st32(s_tm, pk); tmem_st32(s_tm + 32, pk + 32); }
+    } else {
+      uint32_t hi[COLS / 2], lo[COLS / 2];
+      p_chunk_fp8<POLY_MASK, COLS / 2>(sr, ch, c, m, acc, hi, lo);
+      if (ch > 0) {
+        release_chunk(p_full_t + ch - 1);
+      }
+      if constexpr (COLS == 16) {
+        tmem_st8(s_tm + 8 * ch, hi);
+        tmem_st8(s_tm + 32 + 8 * ch, lo);
+      } else if constexpr (COLS == 32) {
+        tmem_st16(s_tm + 16 * ch, hi);
+        tmem_st16(s_tm + 32 + 16 * ch, lo);
+      } else {
+        tmem_st32(s_tm, hi);
+        tmem_st32(s_tm + 32, lo);
+      }
+    }
+  }
+  release_chunk(p_full_t + C::P_CHUNKS - 1);
+  float a, b;
+  f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a, b);
+  return a + b;
+}
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
@@ -131,8 +306,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* kv_full = bars + 1;                  // NSLOT
   uint64_t* kv_empty = kv_full + C::NSLOT;       // NSLOT
   uint64_t* s_full = kv_empty + C::NSLOT;        // Q_TILES
-  uint64_t* p_full = s_full + C::Q_TILES;        // Q_TILES
-  uint64_t* o_done = p_full + C::Q_TILES;        // Q_TILES
+  uint64_t* p_full = s_full + C::Q_TILES;        // Q_TILES x P_CHUNKS
+  uint64_t* o_done = p_full + C::Q_TILES * C::P_CHUNKS;  // Q_TILES
   uint64_t* drain_bar = o_done + C::Q_TILES;     // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
   uint32_t* abort_word = tmem_slot + 1;
@@ -163,7 +338,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     for (int t = 0; t < C::Q_TILES; ++t) {
       mbar_init(s_full + t, 1);
-      mbar_init(p_full + t, 128);
+      for (int c = 0; c < C::P_CHUNKS; ++c) mbar_init(p_full + t * C::P_CHUNKS + c, 128);
       mbar_init(o_done + t, 1);
     }
     mbar_init(drain_bar, 1);
@@ -179,16 +354,28 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const Waiter waiter{abort_word, p.timeout_ns};
+  const Waiter waiter{abort_word, p.timeout_cycles};
 
+  // Each role re-sizes its registers inside its own branch, so the compiler can
+  // give every branch the budget it was granted.
   if (warp == C::PRODUCER_WARP) {
     // ======================= TMA producer =======================
-    if (lane == 0) {
+    // The control warps run their loops with all 32 lanes, so loop state and
+    // addresses stay warp-uniform; one elected lane issues each asynchronous
+    // operation. (A single divergent lane issuing work is starved of issue
+    // slots by the softmax warps that share its scheduler.)
+    regs_decrease<C::REGS_CONTROL>();
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, waiter.wait(bar, parity));
+    };
+    if (elect_one()) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      const uint64_t pol_q = l2_policy_evict_first();
-      const uint64_t pol_kv = l2_policy_evict_last();
+    }
+    const uint64_t pol_q = l2_policy_evict_first();
+    const uint64_t pol_kv = l2_policy_evict_last();
+    if (elect_one()) {
       mbar_arrive_expect_tx(q_full, C::Q_TILES * C::TILE_BYTES);
 #pragma unroll
       for (int t = 0; t < C::Q_TILES; ++t)
@@ -196,120 +383,159 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int c = 0; c < C::CHUNKS; ++c)
           tma_load_3d(smem + C::SMEM_Q + t * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, q_full, c * C::SW_COLS,
                       (qpair * C::Q_TILES + t) * kBlockM, bh, pol_q);
-      const int nloads = 2 * nkv_max;
-      int issued = 0;
-      for (int i = 0; i < nloads; ++i) {
-        const int slot = i % C::NSLOT;
-        if (i >= C::NSLOT) {
-          if (!waiter.wait(kv_empty + slot, ((i / C::NSLOT) - 1) & 1)) {
-            record_timeout();
-            break;
-          }
-        }
-        const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
-        uint8_t* dst = smem + C::SMEM_KV + slot * C::TILE_BYTES;
+    }
+    __syncwarp();
+    const int nloads = 2 * nkv_max;
+    int issued = 0;
+    bool ok = true;
+    for (int i = 0; i < nloads; ++i) {
+      const int slot = i % C::NSLOT;
+      if (i >= C::NSLOT && !(ok = wait_all(kv_empty + slot, ((i / C::NSLOT) - 1) & 1))) break;
+      const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
+      uint8_t* dst = smem + C::SMEM_KV + slot * C::TILE_BYTES;
+      if (elect_one()) {
         mbar_arrive_expect_tx(kv_full + slot, C::TILE_BYTES);
 #pragma unroll
         for (int c = 0; c < C::CHUNKS; ++c)
           tma_load_3d(dst + c * C::CHUNK_BYTES, tm, kv_full + slot, c * C::SW_COLS, (i >> 1) * kBlockN, bh, pol_kv);
-        issued = i + 1;
       }
-      if (waiter.aborted()) {
-        // let every copy still in flight land before shared memory is released
-        drain_wait(q_full, 0, p.timeout_ns);
-        for (int i = max(0, issued - C::NSLOT); i < issued; ++i)
-          drain_wait(kv_full + (i % C::NSLOT), (i / C::NSLOT) & 1, p.timeout_ns);
-      }
+      __syncwarp();
+      issued = i + 1;
+    }
+    if (!ok) {
+      if (lane == 0) record_timeout();
+      // let every copy still in flight land before shared memory is released
+      drain_wait(q_full, 0, p.timeout_cycles);
+      for (int i = max(0, issued - C::NSLOT); i < issued; ++i)
+        drain_wait(kv_full + (i % C::NSLOT), (i / C::NSLOT) & 1, p.timeout_cycles);
     }
     __syncwarp();
   } else if (warp == C::MMA_WARP) {
     // ======================= MMA issuer =======================
-    if (lane == 0) {
-      constexpr uint32_t fmt = C::FP8 ? 0u : 1u;
-      constexpr uint32_t idesc_s = instr_desc(fmt, 128, kBlockN, 0, 0);
-      constexpr uint32_t idesc_o = instr_desc(fmt, 128, C::D, 0, 1);
-      const uint32_t q_base = smem_addr(smem + C::SMEM_Q);
-      const uint32_t kv_base = smem_addr(smem + C::SMEM_KV);
-      bool ok = waiter.wait(q_full, 0);
-      // S_t = Q_t K_j^T over D in UMMA_K steps (K-major operands, 128B swizzle)
-      auto issue_s = [&](int t, uint32_t k_addr) {
-        const uint32_t qa = q_base + t * C::TILE_BYTES;
+    // Warp-uniform loop; one elected lane issues every tcgen05.mma and commit.
+    regs_decrease<C::REGS_CONTROL>();
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, waiter.wait(bar, parity));
+    };
+    auto commit = [&](uint64_t* bar) {
+      if (elect_one()) mma_commit(bar);
+      __syncwarp();
+    };
+    constexpr uint32_t fmt = C::FP8 ? 0u : 1u;
+    constexpr uint32_t idesc_s = instr_desc(fmt, 128, kBlockN, 0, 0);
+    constexpr uint32_t idesc_o = instr_desc(fmt, 128, C::D, 0, 1);
+    // Descriptor words, computed once: per k-step and per slot only the low
+    // word moves (by a compile-time or per-slot constant).
+    constexpr uint32_t hi_kmaj = smem_desc_hi(1024);   // 8 rows x 128 B per swizzle atom
+    constexpr uint32_t hi_mnmaj = smem_desc_hi(1024);
+    const uint32_t q_lo = smem_desc_lo(smem_addr(smem + C::SMEM_Q), 16);
+    const uint32_t k_lo = smem_desc_lo(smem_addr(smem + C::SMEM_KV), 16);
+    const uint32_t v_lo = smem_desc_lo(smem_addr(smem + C::SMEM_KV), C::CHUNK_BYTES);
+    // S_t = Q_t K_j^T over D in UMMA_K steps (K-major operands, 128B swizzle)
+    auto issue_s = [&](int t, int slot) {
+      const uint32_t qa = q_lo + ((t * C::TILE_BYTES) >> 4);
+      const uint32_t ka = k_lo + ((slot * C::TILE_BYTES) >> 4);
+      const uint32_t d_tmem = tmem_base + t * 128;
 #pragma unroll
-        for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
-          const uint32_t off = (kk / (C::SW_COLS / C::UMMA_K)) * C::CHUNK_BYTES + (kk % (C::SW_COLS / C::UMMA_K)) * 32;
-          const uint64_t da = smem_desc(qa + off, 16, 1024);
-          const uint64_t db = smem_desc(k_addr + off, 16, 1024);
+      for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
+        constexpr int per_chunk = C::SW_COLS / C::UMMA_K;
+        const uint32_t off = ((kk / per_chunk) * C::CHUNK_BYTES + (kk % per_chunk) * 32) >> 4;
+        const uint64_t da = smem_desc(qa + off, hi_kmaj);
+        const uint64_t db = smem_desc(ka + off, hi_kmaj);
+        if (elect_one()) {
           if constexpr (C::FP8)
-            mma_f8_ss(tmem_base + t * 128, da, db, idesc_s, kk > 0);
+            mma_f8_ss(d_tmem, da, db, idesc_s, kk > 0);
           else
-            mma_f16_ss(tmem_base + t * 128, da, db, idesc_s, kk > 0);
+            mma_f16_ss(d_tmem, da, db, idesc_s, kk > 0);
         }
-      };
-      // O_t (+)= P_t V_j: P from TMEM (over S_t), V MN-major in shared memory
-      auto issue_pv = [&](int t, uint32_t v_addr, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < C::PV_KSTEPS_TOTAL; ++kk) {
-          const uint64_t db = smem_desc(v_addr + (kk % C::PV_KSTEPS) * C::UMMA_K * 128, C::CHUNK_BYTES, 1024);
-          const uint32_t a_tmem = tmem_base + t * 128 + kk * 8;
-          if constexpr (C::FP8)
-            mma_f8_ts(tmem_base + C::O_COL0 + t * C::D, a_tmem, db, idesc_o, (acc || kk > 0) ? 1u : 0u);
-          else
-            mma_f16_ts(tmem_base + C::O_COL0 + t * C::D, a_tmem, db, idesc_o, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      // K_0: S_t(0) for every tile
-      if (ok && nkv_max > 0) {
-        ok = waiter.wait(kv_full + 0, 0);
-        if (ok) {
-          tc_fence_after();
-#pragma unroll
-          for (int t = 0; t < C::Q_TILES; ++t)
-            if (nkv[t] > 0) {
-              issue_s(t, kv_base);
-              mma_commit(s_full + t);
-            }
-          mma_commit(kv_empty + 0);
-        }
+        __syncwarp();
       }
-      for (int j = 0; ok && j < nkv_max; ++j) {
-        const int vi = 2 * j + 1, ki = 2 * j + 2;
-        const int vslot = vi % C::NSLOT, kslot = ki % C::NSLOT;
-        bool v_ready = false, k_ready = false, any_s = false;
+    };
+    // O_t (+)= P_t V_j for the keys of P chunk c: P from TMEM (over S_t), V
+    // MN-major in shared memory. bf16: two K=16 steps per chunk; FP8: the hi
+    // and the lo step of the chunk's 32 keys.
+    auto issue_pv_chunk = [&](int t, int slot, int c, bool acc) {
+      const uint32_t va = v_lo + ((slot * C::TILE_BYTES) >> 4);
+      const uint32_t o_tmem = tmem_base + C::O_COL0 + t * C::D;
+      const uint32_t p_tmem = tmem_base + t * 128;
+      constexpr int STEPS = C::PV_KSTEPS / C::P_CHUNKS;   // K steps per chunk per term
 #pragma unroll
-        for (int t = 0; t < C::Q_TILES; ++t) {
-          if (j >= nkv[t]) continue;
-          if (!(ok = waiter.wait(p_full + t, j & 1))) break;
-          if (!v_ready) {
-            if (!(ok = waiter.wait(kv_full + vslot, (vi / C::NSLOT) & 1))) break;
-            v_ready = true;
+      for (int term = 0; term < (C::FP8 ? 2 : 1); ++term)
+#pragma unroll
+        for (int i = 0; i < STEPS; ++i) {
+          const int kv = c * STEPS + i;                     // K step within V
+          const int kk = term * C::PV_KSTEPS + kv;          // K step within [hi | lo]
+          const uint64_t db = smem_desc(va + ((kv * C::UMMA_K * 128) >> 4), hi_mnmaj);
+          const uint32_t accum = (acc || term > 0 || i > 0) ? 1u : 0u;
+          if (elect_one()) {
+            if constexpr (C::FP8)
+              mma_f8_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum);
+            else
+              mma_f16_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum);
           }
+          __syncwarp();
+        }
+    };
+    bool ok = wait_all(q_full, 0);
+    // K_0: S_t(0) for every tile
+    if (ok && nkv_max > 0) {
+      ok = wait_all(kv_full + 0, 0);
+      if (ok) {
+        tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < C::Q_TILES; ++t)
+          if (nkv[t] > 0) {
+            issue_s(t, 0);
+            commit(s_full + t);
+          }
+        commit(kv_empty + 0);
+      }
+    }
+    for (int j = 0; ok && j < nkv_max; ++j) {
+      const int vi = 2 * j + 1, ki = 2 * j + 2;
+      const int vslot = vi % C::NSLOT, kslot = ki % C::NSLOT;
+      bool v_ready = false, k_ready = false, any_s = false;
+#pragma unroll
+      for (int t = 0; t < C::Q_TILES; ++t) {
+        if (j >= nkv[t]) continue;
+        if (!v_ready) {
+          if (!(ok = wait_all(kv_full + vslot, (vi / C::NSLOT) & 1))) break;
+          v_ready = true;
+        }
+#pragma unroll
+        for (int c = 0; c < C::P_CHUNKS; ++c) {
+          if (!(ok = wait_all(p_full + t * C::P_CHUNKS + c, j & 1))) break;
           tc_fence_after();
-          issue_pv(t, kv_base + vslot * C::TILE_BYTES, j > 0);
-          if (j + 1 < nkv[t]) {
-            if (!k_ready) {
-              if (!(ok = waiter.wait(kv_full + kslot, (ki / C::NSLOT) & 1))) break;
-              k_ready = true;
-              tc_fence_after();
-            }
-            issue_s(t, kv_base + kslot * C::TILE_BYTES);
-            mma_commit(s_full + t);
-            any_s = true;
-          } else {
-            mma_commit(o_done + t);
-          }
+          issue_pv_chunk(t, vslot, c, j > 0 || c > 0);
         }
         if (!ok) break;
-        mma_commit(kv_empty + vslot);
-        if (any_s) mma_commit(kv_empty + kslot);
+        if (j + 1 < nkv[t]) {
+          if (!k_ready) {
+            if (!(ok = wait_all(kv_full + kslot, (ki / C::NSLOT) & 1))) break;
+            k_ready = true;
+            tc_fence_after();
+          }
+          issue_s(t, kslot);
+          commit(s_full + t);
+          any_s = true;
+        } else {
+          commit(o_done + t);
+        }
       }
-      if (!ok) record_timeout();
-      // every MMA this thread issued completes before TMEM can be released
-      mma_commit(drain_bar);
-      drain_wait(drain_bar, 0, p.timeout_ns);
+      if (!ok) break;
+      commit(kv_empty + vslot);
+      if (any_s) commit(kv_empty + kslot);
     }
+    if (!ok && lane == 0) record_timeout();
+    // every MMA this warp issued completes before TMEM can be released
+    commit(drain_bar);
+    drain_wait(drain_bar, 0, p.timeout_cycles);
     __syncwarp();
+  } else if (warp > C::MMA_WARP) {
+    regs_decrease<C::REGS_CONTROL>();  // idle warps of the control warpgroup
   } else {
     // ======================= softmax groups =======================
+    regs_increase<C::REGS_SOFTMAX>();
     const int t = warp >> 2;                 // Q tile of this group
     const int wq = warp & 3;                 // lane quarter of TMEM this warp may access
     const int r = wq * 32 + lane;            // row inside the tile
@@ -319,12 +545,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t s_tm = tmem_base + lane_off + t * 128;
     const uint32_t o_tm = tmem_base + lane_off + C::O_COL0 + t * C::D;
     const int T = (p.N + kBlockN - 1) / kBlockN;   // tiles per head (FP8 scales)
+    int nkv_t = nkv[0];                             // (no dynamic indexing: keeps nkv in registers)
+#pragma unroll
+    for (int i = 1; i < C::Q_TILES; ++i)
+      if (t == i) nkv_t = nkv[i];
 
     float m_run = __int_as_float(0xff800000u);   // running max of scale*log2(e)*s, log2 units
     float l_run = 0.f;         // running normaliser, relative to 2^m_run
     float q_sc = 1.f, v_max = 1.f;
     if constexpr (C::FP8) {
-      if (nkv[t] > 0) {
+      if (nkv_t > 0) {
         q_sc = p.q_scale[bh * T + qb];
         float vm = 0.f;
         for (int i = 0; i < T; ++i) vm = fmaxf(vm, p.v_scale[bh * T + i]);
@@ -332,7 +562,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     }
     bool ok = true;
-    for (int j = 0; j < nkv[t]; ++j) {
+    for (int j = 0; j < nkv_t; ++j) {
       // TMEM loads/stores below are warp-collective: the whole warp goes on or stops
       ok = __all_sync(0xffffffffu, waiter.wait(s_full + t, j & 1));
       if (!ok) break;
@@ -343,61 +573,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tmem_ld32(s_tm + 64, sr + 64);
       tmem_ld32(s_tm + 96, sr + 96);
       tmem_ld_wait<128>(sr);
-
-      float c = p.scale_log2;
-      float v_log2_ratio = 0.f;
+      float c = p.scale_log2, v_log2_ratio = 0.f;
       if constexpr (C::FP8) {
         c *= q_sc * p.k_scale[bh * T + j];
         v_log2_ratio = __log2f(p.v_scale[bh * T + j] / v_max);
       }
       // masking: causal diagonal block and the ragged last key block
-      if (j == nkv[t] - 1 && (p.causal || (p.N % kBlockN) != 0)) {
+      const bool masked = (j == nkv_t - 1) && (p.causal || (p.N % kBlockN) != 0);
+      if (masked) {
         const int limit = (p.causal ? min(row, p.N - 1) : p.N - 1) - j * kBlockN;  // last visible column
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (i > limit) sr[i] = 0xff800000u;  // -inf
       }
-      float mx = __int_as_float(0xff800000u);
-#pragma unroll
-      for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
-      const float m_blk = mx * c;
+      const float m_blk = row_max128(sr) * c;
       float m_use = m_run;
       if (m_blk - m_run > C::RESCALE_THRESHOLD) m_use = m_blk;
-      const float alpha = ex2_approx(m_run - m_use);     // 0 on the first block
       // exponent offset: FP8 folds the V tile scale ratio and a 2^8 pre-scale in
       const float m_exp = C::FP8 ? (m_use - v_log2_ratio - C::P_PRESCALE_LOG2) : m_use;
-      float sum = 0.f;
-      uint32_t pk[C::P_COLS];
-      if constexpr (!C::FP8) {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[2 * i]), c, -m_exp));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[2 * i + 1]), c, -m_exp));
-          sum += p0 + p1;
-          pk[i] = pack_bf16x2(p0, p1);
-        }
-      } else {
-        // P = hi + lo, both E4M3: hi = e4m3(p), lo = e4m3(p - hi) (residual in f16)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[4 * i]), c, -m_exp));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[4 * i + 1]), c, -m_exp));
-          const float p2 = ex2_approx(fmaf(__uint_as_float(sr[4 * i + 2]), c, -m_exp));
-          const float p3 = ex2_approx(fmaf(__uint_as_float(sr[4 * i + 3]), c, -m_exp));
-          sum += (p0 + p1) + (p2 + p3);
-          const uint32_t h01 = pack_f16x2(p0, p1), h23 = pack_f16x2(p2, p3);
-          const uint16_t hi01 = e4m3x2_from_f16x2(h01), hi23 = e4m3x2_from_f16x2(h23);
-          const uint16_t lo01 = e4m3x2_from_f16x2(hsub2_u32(h01, f16x2_from_e4m3x2(hi01)));
-          const uint16_t lo23 = e4m3x2_from_f16x2(hsub2_u32(h23, f16x2_from_e4m3x2(hi23)));
-          pk[i] = static_cast<uint32_t>(hi01) | (static_cast<uint32_t>(hi23) << 16);
-          pk[32 + i] = static_cast<uint32_t>(lo01) | (static_cast<uint32_t>(lo23) << 16);
-        }
-        // back to the units of 2^m_use
-        sum *= ex2_approx(-v_log2_ratio - C::P_PRESCALE_LOG2);
-      }
+      const bool moved = m_use != m_run;
+      // 2^(m_run - m_use); 0 on the first block
+      const float alpha = moved ? ex2_approx(m_run - m_use) : 1.f;
       // O_t rescale when this warp moved its maximum (O_t already holds every
-      // earlier P V: the commit behind s_full covers them)
-      if (j > 0 && __any_sync(0xffffffffu, m_use != m_run)) {
+      // earlier P V: the commit behind s_full covers them); it must land before
+      // the first P chunk of this block is released to the MMA.
+      if (j > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll
         for (int cb = 0; cb < C::D; cb += 32) {
           uint32_t ov[32];
@@ -408,18 +608,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tmem_st32(o_tm + cb, ov);
         }
       }
-      // P_t over the first columns of S_t
-      tmem_st32(s_tm + 0, pk);
-      tmem_st32(s_tm + 32, pk + 32);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(p_full + t);
+      // P_t over the first columns of S_t, chunk by chunk; masked blocks keep
+      // every exponential on MUFU (exact zeros for -inf)
+      uint64_t* pf = p_full + t * C::P_CHUNKS;
+      float sum = masked ? p_row_to_tmem<C, 0u>(sr, c, m_exp, s_tm, pf)
+                         : p_row_to_tmem<C, C::POLY_MASK>(sr, c, m_exp, s_tm, pf);
+      if constexpr (C::FP8) sum *= ex2_approx(-v_log2_ratio - C::P_PRESCALE_LOG2);  // units of 2^m_use
       l_run = l_run * alpha + sum;
       m_run = m_use;
     }
     if (!ok) record_timeout();
     // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2
-    if (ok && nkv[t] > 0) {
+    if (ok && nkv_t > 0) {
       if (__all_sync(0xffffffffu, waiter.wait(o_done + t, 0))) {
         tc_fence_after();
         float inv_l = 1.f / l_run;

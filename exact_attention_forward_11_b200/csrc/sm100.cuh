@@ -13,12 +13,6 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count) : "memory");
@@ -49,22 +43,33 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded waiting. Every wait of a CTA shares one abort word in shared memory:
-// the first wait that runs past `limit_ns` sets it (and the caller records the
-// failure in global memory); every later wait of the CTA then returns false at
-// once, so all roles leave their loops and the CTA exits instead of hanging.
+// the first wait that runs past its cycle budget sets it (and the caller records
+// the failure in global memory); every later wait of the CTA then returns false
+// soon after, so all roles leave their loops and the CTA exits instead of
+// hanging. The barrier is polled back to back; the SM cycle counter and the
+// abort word are only read every 64 polls, so a completed phase is seen within a
+// few tens of cycles.
+__device__ __forceinline__ uint64_t sm_clock() {
+  uint64_t c;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(c));
+  return c;
+}
+
 struct Waiter {
   volatile uint32_t* abort_flag;  // shared memory
-  uint64_t limit_ns;
+  uint64_t limit_cycles;
 
   __device__ __forceinline__ bool wait(uint64_t* bar, uint32_t parity) const {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_timer_ns();
-    while (true) {
+    const uint64_t t0 = sm_clock();
+    for (uint32_t it = 1;; ++it) {
       if (mbar_try_wait(bar, parity)) return true;
-      if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > limit_ns) {
-        *abort_flag = 1u;
-        return false;
+      if ((it & 63u) == 0u) {
+        if (*abort_flag) return false;
+        if (sm_clock() - t0 > limit_cycles) {
+          *abort_flag = 1u;
+          return false;
+        }
       }
     }
   }
@@ -171,22 +176,32 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       B200_W8(0), B200_W8(8)
       : "memory");
 }
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), B200_W8(0)
+               : "memory");
+}
 #undef B200_W8
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- MMA
-// Shared-memory matrix descriptor (tcgen05 format): start address, leading and
-// stride byte offsets (all >> 4), descriptor version 1, swizzle mode.
-enum : uint64_t { kSwizzle128B = 2 };
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= 1ull << 46;                  // version
-  d |= kSwizzle128B << 61;          // 128-byte swizzle
+// Shared-memory matrix descriptor (tcgen05 format), split in two 32-bit words:
+//   low : start address >> 4 (bits 0-13), leading byte offset >> 4 (bits 16-29)
+//   high: stride byte offset >> 4 (bits 32-45), version 1 (bit 46), swizzle
+//         mode 128B = 2 (bits 61-63)
+// Moving the start address by a multiple of 16 bytes inside a tile is a plain
+// add on the low word (the 14-bit field cannot carry: shared addresses < 256 KB).
+enum : uint32_t { kSwizzle128B = 2 };
+__host__ __device__ constexpr uint32_t smem_desc_hi(uint32_t sbo_bytes) {
+  return ((sbo_bytes >> 4) & 0x3FFFu) | (1u << 14) | (kSwizzle128B << 29);
+}
+__device__ __forceinline__ uint32_t smem_desc_lo(uint32_t saddr, uint32_t lbo_bytes) {
+  return ((saddr >> 4) & 0x3FFFu) | (((lbo_bytes >> 4) & 0x3FFFu) << 16);
+}
+__device__ __forceinline__ uint64_t smem_desc(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
   return d;
 }
 
@@ -269,6 +284,64 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+
+// ---------------------------------------------------------------- warp election
+// True on exactly one lane of a fully active warp (elect.sync picks the same
+// leader every time for the same set of active lanes, so tcgen05 operations and
+// the commits that track them all come from one thread).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+// ---------------------------------------------------------------- registers
+// Per-warpgroup register re-allocation; every warp of the warpgroup executes it.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ---------------------------------------------------------------- packed fp32
+// (Measured on B200: fma.rn.f32x2 competes with MUFU ex2 for issue, add/sub
+// f32x2 and scalar FMA do not; the softmax therefore multiplies with scalar FMAs
+// and uses the packed forms only for additions.)
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 // fp32 pair -> f16x2 (element 0 in the low half)
