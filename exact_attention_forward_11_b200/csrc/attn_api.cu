@@ -57,6 +57,18 @@ bool encode_qkv_map(CUtensorMap* map, const void* base, bool fp8, int d, int N, 
   return r == CUDA_SUCCESS;
 }
 
+// Number of SMs of the current device (cached per device ordinal).
+int sm_count() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
+  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev < 64) cache[dev] = n;
+  return n;
+}
+
 attn_status check_shape(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
   const long long rows = static_cast<long long>(B) * H * N;
@@ -89,7 +101,12 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.k_scale = ks;
   p.v_scale = vs;
   p.timeout_cycles = kWaitLimitCycles;
-  kern<<<p.num_units, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  // persistent grid: one CTA per SM (shared memory and TMEM allow one), each
+  // walking the units blockIdx.x, blockIdx.x + gridDim.x, ...
+  const int sms = sm_count();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  const int grid = p.num_units < sms ? p.num_units : sms;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 

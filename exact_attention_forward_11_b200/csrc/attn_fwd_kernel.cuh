@@ -110,7 +110,7 @@ struct FwdCfg {
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_KV = SMEM_Q + Q_TILES * TILE_BYTES;
   static constexpr int SMEM_BAR = SMEM_KV + NSLOT * TILE_BYTES;
-  static constexpr int NUM_BARS = 1 + 2 * NSLOT + (2 + P_CHUNKS) * Q_TILES + 1;
+  static constexpr int NUM_BARS = 2 + 2 * NSLOT + (2 + P_CHUNKS) * Q_TILES + 1;
   static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
 };
@@ -294,6 +294,35 @@ __device__ __forceinline__ float p_row_to_tmem(const uint32_t (&sr)[128], float 
   return a + b;
 }
 
+// Work unit u of a launch: the pair of Q tiles `qpair` of head `bh`. Units are
+// numbered heaviest causal pairs first (u / BH counts down the pairs). A
+// persistent CTA b takes one unit per round k in snake order: unit
+// k*G + b on even rounds and k*G + G-1-b on odd rounds (G = gridDim.x), so a CTA
+// that got one of the heavier units of a round gets one of the lighter ones in
+// the next: the causal work per CTA balances without a shared work counter.
+__device__ __forceinline__ int unit_of_round(int k) {
+  const int base = k * static_cast<int>(gridDim.x);
+  return (k & 1) ? base + static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x)
+                 : base + static_cast<int>(blockIdx.x);
+}
+
+template <class C>
+struct UnitInfo {
+  int qpair, bh, nkv_max;
+  int nkv[C::Q_TILES];
+  __device__ __forceinline__ UnitInfo(const FwdParams& p, int u, int QB, int NPAIR) {
+    qpair = NPAIR - 1 - u / p.BH;
+    bh = u % p.BH;
+    nkv_max = 0;
+#pragma unroll
+    for (int t = 0; t < C::Q_TILES; ++t) {
+      const int qb = qpair * C::Q_TILES + t;
+      nkv[t] = (qb >= QB) ? 0 : (p.causal ? qb + 1 : QB);
+      nkv_max = max(nkv_max, nkv[t]);
+    }
+  }
+};
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -309,29 +338,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* p_full = s_full + C::Q_TILES;        // Q_TILES x P_CHUNKS
   uint64_t* o_done = p_full + C::Q_TILES * C::P_CHUNKS;  // Q_TILES
   uint64_t* drain_bar = o_done + C::Q_TILES;     // 1
+  uint64_t* q_empty = drain_bar + 1;             // 1
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
   uint32_t* abort_word = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work unit: (head bh, pair of Q tiles); heavy causal units first
   const int QB = (p.N + kBlockM - 1) / kBlockM;
   const int NPAIR = (QB + C::Q_TILES - 1) / C::Q_TILES;
-  const int unit = blockIdx.x;
-  const int qpair = NPAIR - 1 - unit / p.BH;
-  const int bh = unit % p.BH;
-  int nkv[C::Q_TILES];
-  int nkv_max = 0;
-#pragma unroll
-  for (int t = 0; t < C::Q_TILES; ++t) {
-    const int qb = qpair * C::Q_TILES + t;
-    nkv[t] = (qb >= QB) ? 0 : (p.causal ? qb + 1 : QB);
-    nkv_max = max(nkv_max, nkv[t]);
-  }
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(kv_full + i, 1);
       mbar_init(kv_empty + i, 1);
@@ -356,8 +374,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   const Waiter waiter{abort_word, p.timeout_cycles};
 
-  // Each role re-sizes its registers inside its own branch, so the compiler can
-  // give every branch the budget it was granted.
+  // Every barrier phase below is a running count over all units this CTA
+  // processes (the pipeline is not reset between units). Each role re-sizes
+  // its registers inside its own branch, so the compiler can give every branch
+  // the budget it was granted.
   if (warp == C::PRODUCER_WARP) {
     // ======================= TMA producer =======================
     // The control warps run their loops with all 32 lanes, so loop state and
@@ -375,38 +395,46 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     const uint64_t pol_q = l2_policy_evict_first();
     const uint64_t pol_kv = l2_policy_evict_last();
-    if (elect_one()) {
-      mbar_arrive_expect_tx(q_full, C::Q_TILES * C::TILE_BYTES);
-#pragma unroll
-      for (int t = 0; t < C::Q_TILES; ++t)
-#pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(smem + C::SMEM_Q + t * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, q_full, c * C::SW_COLS,
-                      (qpair * C::Q_TILES + t) * kBlockM, bh, pol_q);
-    }
-    __syncwarp();
-    const int nloads = 2 * nkv_max;
-    int issued = 0;
+    uint32_t g = 0;        // K/V tile loads issued so far (slot g % NSLOT, phase g / NSLOT)
+    int q_loads = 0;       // Q loads issued so far (phase of q_full)
     bool ok = true;
-    for (int i = 0; i < nloads; ++i) {
-      const int slot = i % C::NSLOT;
-      if (i >= C::NSLOT && !(ok = wait_all(kv_empty + slot, ((i / C::NSLOT) - 1) & 1))) break;
-      const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
-      uint8_t* dst = smem + C::SMEM_KV + slot * C::TILE_BYTES;
+    for (int k = 0; ok && k * static_cast<int>(gridDim.x) < p.num_units; ++k) {
+      const int u = unit_of_round(k);
+      if (u >= p.num_units) continue;
+      const UnitInfo<C> w(p, u, QB, NPAIR);
+      // Q is reused by the previous unit's S MMAs until they complete
+      if (q_loads > 0 && !(ok = wait_all(q_empty, (q_loads - 1) & 1))) break;
       if (elect_one()) {
-        mbar_arrive_expect_tx(kv_full + slot, C::TILE_BYTES);
+        mbar_arrive_expect_tx(q_full, C::Q_TILES * C::TILE_BYTES);
 #pragma unroll
-        for (int c = 0; c < C::CHUNKS; ++c)
-          tma_load_3d(dst + c * C::CHUNK_BYTES, tm, kv_full + slot, c * C::SW_COLS, (i >> 1) * kBlockN, bh, pol_kv);
+        for (int t = 0; t < C::Q_TILES; ++t)
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_3d(smem + C::SMEM_Q + t * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, q_full, c * C::SW_COLS,
+                        (w.qpair * C::Q_TILES + t) * kBlockM, w.bh, pol_q);
       }
       __syncwarp();
-      issued = i + 1;
+      ++q_loads;
+      for (int i = 0; i < 2 * w.nkv_max; ++i, ++g) {
+        const uint32_t slot = g % C::NSLOT;
+        if (g >= C::NSLOT && !(ok = wait_all(kv_empty + slot, ((g / C::NSLOT) - 1) & 1))) break;
+        const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;
+        uint8_t* dst = smem + C::SMEM_KV + slot * C::TILE_BYTES;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(kv_full + slot, C::TILE_BYTES);
+#pragma unroll
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_3d(dst + c * C::CHUNK_BYTES, tm, kv_full + slot, c * C::SW_COLS, (i >> 1) * kBlockN, w.bh,
+                        pol_kv);
+        }
+        __syncwarp();
+      }
     }
     if (!ok) {
       if (lane == 0) record_timeout();
       // let every copy still in flight land before shared memory is released
-      drain_wait(q_full, 0, p.timeout_cycles);
-      for (int i = max(0, issued - C::NSLOT); i < issued; ++i)
+      if (q_loads > 0) drain_wait(q_full, (q_loads - 1) & 1, p.timeout_cycles);
+      for (uint32_t i = (g > C::NSLOT ? g - C::NSLOT : 0); i < g; ++i)
         drain_wait(kv_full + (i % C::NSLOT), (i / C::NSLOT) & 1, p.timeout_cycles);
     }
     __syncwarp();
@@ -432,7 +460,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t k_lo = smem_desc_lo(smem_addr(smem + C::SMEM_KV), 16);
     const uint32_t v_lo = smem_desc_lo(smem_addr(smem + C::SMEM_KV), C::CHUNK_BYTES);
     // S_t = Q_t K_j^T over D in UMMA_K steps (K-major operands, 128B swizzle)
-    auto issue_s = [&](int t, int slot) {
+    auto issue_s = [&](int t, uint32_t slot) {
       const uint32_t qa = q_lo + ((t * C::TILE_BYTES) >> 4);
       const uint32_t ka = k_lo + ((slot * C::TILE_BYTES) >> 4);
       const uint32_t d_tmem = tmem_base + t * 128;
@@ -452,9 +480,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     };
     // O_t (+)= P_t V_j for the keys of P chunk c: P from TMEM (over S_t), V
-    // MN-major in shared memory. bf16: two K=16 steps per chunk; FP8: the hi
-    // and the lo step of the chunk's 32 keys.
-    auto issue_pv_chunk = [&](int t, int slot, int c, bool acc) {
+    // MN-major in shared memory. bf16: K=16 steps; FP8: the hi and the lo steps
+    // of the chunk's keys.
+    auto issue_pv_chunk = [&](int t, uint32_t slot, int c, bool acc) {
       const uint32_t va = v_lo + ((slot * C::TILE_BYTES) >> 4);
       const uint32_t o_tmem = tmem_base + C::O_COL0 + t * C::D;
       const uint32_t p_tmem = tmem_base + t * 128;
@@ -476,55 +504,68 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           __syncwarp();
         }
     };
-    bool ok = wait_all(q_full, 0);
-    // K_0: S_t(0) for every tile
-    if (ok && nkv_max > 0) {
-      ok = wait_all(kv_full + 0, 0);
-      if (ok) {
-        tc_fence_after();
+    uint32_t g = 0;                       // K/V tiles consumed so far (same count as the producer's)
+    uint32_t pc[C::Q_TILES];              // blocks of P consumed per tile (p_full phases)
 #pragma unroll
-        for (int t = 0; t < C::Q_TILES; ++t)
-          if (nkv[t] > 0) {
-            issue_s(t, 0);
-            commit(s_full + t);
-          }
-        commit(kv_empty + 0);
-      }
-    }
-    for (int j = 0; ok && j < nkv_max; ++j) {
-      const int vi = 2 * j + 1, ki = 2 * j + 2;
-      const int vslot = vi % C::NSLOT, kslot = ki % C::NSLOT;
-      bool v_ready = false, k_ready = false, any_s = false;
+    for (int t = 0; t < C::Q_TILES; ++t) pc[t] = 0;
+    int units = 0;
+    bool ok = true;
+    for (int k = 0; ok && k * static_cast<int>(gridDim.x) < p.num_units; ++k) {
+      const int u = unit_of_round(k);
+      if (u >= p.num_units) continue;
+      const UnitInfo<C> w(p, u, QB, NPAIR);
+      if (!(ok = wait_all(q_full, units & 1))) break;
+      // K_0: S_t(0) for every tile (issued after the previous unit's last P V on
+      // this thread, so it overwrites that P only after it has been read)
+      if (!(ok = wait_all(kv_full + (g % C::NSLOT), (g / C::NSLOT) & 1))) break;
+      tc_fence_after();
 #pragma unroll
-      for (int t = 0; t < C::Q_TILES; ++t) {
-        if (j >= nkv[t]) continue;
-        if (!v_ready) {
-          if (!(ok = wait_all(kv_full + vslot, (vi / C::NSLOT) & 1))) break;
-          v_ready = true;
+      for (int t = 0; t < C::Q_TILES; ++t)
+        if (w.nkv[t] > 0) {
+          issue_s(t, g % C::NSLOT);
+          commit(s_full + t);
         }
+      commit(kv_empty + (g % C::NSLOT));
+      if (w.nkv_max == 1) commit(q_empty);   // the unit's last S MMAs are issued
+      for (int j = 0; ok && j < w.nkv_max; ++j) {
+        const uint32_t vg = g + 2 * j + 1, kg = g + 2 * j + 2;
+        const uint32_t vslot = vg % C::NSLOT, kslot = kg % C::NSLOT;
+        bool v_ready = false, k_ready = false, any_s = false;
 #pragma unroll
-        for (int c = 0; c < C::P_CHUNKS; ++c) {
-          if (!(ok = wait_all(p_full + t * C::P_CHUNKS + c, j & 1))) break;
-          tc_fence_after();
-          issue_pv_chunk(t, vslot, c, j > 0 || c > 0);
+        for (int t = 0; t < C::Q_TILES; ++t) {
+          if (j >= w.nkv[t]) continue;
+          if (!v_ready) {
+            if (!(ok = wait_all(kv_full + vslot, (vg / C::NSLOT) & 1))) break;
+            v_ready = true;
+          }
+#pragma unroll
+          for (int c = 0; c < C::P_CHUNKS; ++c) {
+            if (!(ok = wait_all(p_full + t * C::P_CHUNKS + c, pc[t] & 1))) break;
+            tc_fence_after();
+            issue_pv_chunk(t, vslot, c, j > 0 || c > 0);
+          }
+          if (!ok) break;
+          ++pc[t];
+          if (j + 1 < w.nkv[t]) {
+            if (!k_ready) {
+              if (!(ok = wait_all(kv_full + kslot, (kg / C::NSLOT) & 1))) break;
+              k_ready = true;
+              tc_fence_after();
+            }
+            issue_s(t, kslot);
+            commit(s_full + t);
+            any_s = true;
+          } else {
+            commit(o_done + t);
+          }
         }
         if (!ok) break;
-        if (j + 1 < nkv[t]) {
-          if (!k_ready) {
-            if (!(ok = wait_all(kv_full + kslot, (ki / C::NSLOT) & 1))) break;
-            k_ready = true;
-            tc_fence_after();
-          }
-          issue_s(t, kslot);
-          commit(s_full + t);
-          any_s = true;
-        } else {
-          commit(o_done + t);
-        }
+        commit(kv_empty + vslot);
+        if (any_s) commit(kv_empty + kslot);
+        if (any_s && j + 2 == w.nkv_max) commit(q_empty);   // the unit's last S MMAs are issued
       }
-      if (!ok) break;
-      commit(kv_empty + vslot);
-      if (any_s) commit(kv_empty + kslot);
+      g += 2 * w.nkv_max;
+      ++units;
     }
     if (!ok && lane == 0) record_timeout();
     // every MMA this warp issued completes before TMEM can be released
@@ -539,115 +580,122 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int t = warp >> 2;                 // Q tile of this group
     const int wq = warp & 3;                 // lane quarter of TMEM this warp may access
     const int r = wq * 32 + lane;            // row inside the tile
-    const int qb = qpair * C::Q_TILES + t;
-    const int row = qb * kBlockM + r;        // query row inside the head
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t s_tm = tmem_base + lane_off + t * 128;
     const uint32_t o_tm = tmem_base + lane_off + C::O_COL0 + t * C::D;
     const int T = (p.N + kBlockN - 1) / kBlockN;   // tiles per head (FP8 scales)
-    int nkv_t = nkv[0];                             // (no dynamic indexing: keeps nkv in registers)
+    uint32_t sc = 0;                               // S_t completions consumed (s_full phases)
+    uint32_t oc = 0;                               // O_t completions consumed (o_done phases)
+    bool ok = true;
+    for (int k = 0; ok && k * static_cast<int>(gridDim.x) < p.num_units; ++k) {
+      const int u = unit_of_round(k);
+      if (u >= p.num_units) continue;
+      const UnitInfo<C> w(p, u, QB, NPAIR);
+      int nkv_t = w.nkv[0];                        // (no dynamic indexing: keeps nkv in registers)
 #pragma unroll
-    for (int i = 1; i < C::Q_TILES; ++i)
-      if (t == i) nkv_t = nkv[i];
-
-    float m_run = __int_as_float(0xff800000u);   // running max of scale*log2(e)*s, log2 units
-    float l_run = 0.f;         // running normaliser, relative to 2^m_run
-    float q_sc = 1.f, v_max = 1.f;
-    if constexpr (C::FP8) {
-      if (nkv_t > 0) {
+      for (int i = 1; i < C::Q_TILES; ++i)
+        if (t == i) nkv_t = w.nkv[i];
+      if (nkv_t == 0) continue;
+      const int bh = w.bh;
+      const int qb = w.qpair * C::Q_TILES + t;
+      const int row = qb * kBlockM + r;            // query row inside the head
+      float m_run = __int_as_float(0xff800000u);   // running max of scale*log2(e)*s, log2 units
+      float l_run = 0.f;                           // running normaliser, relative to 2^m_run
+      float q_sc = 1.f, v_max = 1.f;
+      if constexpr (C::FP8) {
         q_sc = p.q_scale[bh * T + qb];
         float vm = 0.f;
         for (int i = 0; i < T; ++i) vm = fmaxf(vm, p.v_scale[bh * T + i]);
         v_max = vm > 0.f ? vm : 1.f;
       }
-    }
-    bool ok = true;
-    for (int j = 0; j < nkv_t; ++j) {
-      // TMEM loads/stores below are warp-collective: the whole warp goes on or stops
-      ok = __all_sync(0xffffffffu, waiter.wait(s_full + t, j & 1));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sr[128];
-      tmem_ld32(s_tm + 0, sr + 0);
-      tmem_ld32(s_tm + 32, sr + 32);
-      tmem_ld32(s_tm + 64, sr + 64);
-      tmem_ld32(s_tm + 96, sr + 96);
-      tmem_ld_wait<128>(sr);
-      float c = p.scale_log2, v_log2_ratio = 0.f;
-      if constexpr (C::FP8) {
-        c *= q_sc * p.k_scale[bh * T + j];
-        v_log2_ratio = __log2f(p.v_scale[bh * T + j] / v_max);
-      }
-      // masking: causal diagonal block and the ragged last key block
-      const bool masked = (j == nkv_t - 1) && (p.causal || (p.N % kBlockN) != 0);
-      if (masked) {
-        const int limit = (p.causal ? min(row, p.N - 1) : p.N - 1) - j * kBlockN;  // last visible column
-#pragma unroll
-        for (int i = 0; i < 128; ++i)
-          if (i > limit) sr[i] = 0xff800000u;  // -inf
-      }
-      const float m_blk = row_max128(sr) * c;
-      float m_use = m_run;
-      if (m_blk - m_run > C::RESCALE_THRESHOLD) m_use = m_blk;
-      // exponent offset: FP8 folds the V tile scale ratio and a 2^8 pre-scale in
-      const float m_exp = C::FP8 ? (m_use - v_log2_ratio - C::P_PRESCALE_LOG2) : m_use;
-      const bool moved = m_use != m_run;
-      // 2^(m_run - m_use); 0 on the first block
-      const float alpha = moved ? ex2_approx(m_run - m_use) : 1.f;
-      // O_t rescale when this warp moved its maximum (O_t already holds every
-      // earlier P V: the commit behind s_full covers them); it must land before
-      // the first P chunk of this block is released to the MMA.
-      if (j > 0 && __any_sync(0xffffffffu, moved)) {
-#pragma unroll
-        for (int cb = 0; cb < C::D; cb += 32) {
-          uint32_t ov[32];
-          tmem_ld32(o_tm + cb, ov);
-          tmem_ld_wait<32>(ov);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-          tmem_st32(o_tm + cb, ov);
-        }
-      }
-      // P_t over the first columns of S_t, chunk by chunk; masked blocks keep
-      // every exponential on MUFU (exact zeros for -inf)
-      uint64_t* pf = p_full + t * C::P_CHUNKS;
-      float sum = masked ? p_row_to_tmem<C, 0u>(sr, c, m_exp, s_tm, pf)
-                         : p_row_to_tmem<C, C::POLY_MASK>(sr, c, m_exp, s_tm, pf);
-      if constexpr (C::FP8) sum *= ex2_approx(-v_log2_ratio - C::P_PRESCALE_LOG2);  // units of 2^m_use
-      l_run = l_run * alpha + sum;
-      m_run = m_use;
-    }
-    if (!ok) record_timeout();
-    // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2
-    if (ok && nkv_t > 0) {
-      if (__all_sync(0xffffffffu, waiter.wait(o_done + t, 0))) {
+      for (int j = 0; j < nkv_t; ++j) {
+        // TMEM loads/stores below are warp-collective: the whole warp goes on or stops
+        ok = __all_sync(0xffffffffu, waiter.wait(s_full + t, sc & 1));
+        if (!ok) break;
+        ++sc;
         tc_fence_after();
-        float inv_l = 1.f / l_run;
-        if constexpr (C::FP8) inv_l *= v_max * 0.00390625f;  // undo the V ratio and 2^8 pre-scale
-        const bool in_range = row < p.N;
-        __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (in_range ? row : 0)) * C::D;
+        uint32_t sr[128];
+        tmem_ld32(s_tm + 0, sr + 0);
+        tmem_ld32(s_tm + 32, sr + 32);
+        tmem_ld32(s_tm + 64, sr + 64);
+        tmem_ld32(s_tm + 96, sr + 96);
+        tmem_ld_wait<128>(sr);
+        float c = p.scale_log2, v_log2_ratio = 0.f;
+        if constexpr (C::FP8) {
+          c *= q_sc * p.k_scale[bh * T + j];
+          v_log2_ratio = __log2f(p.v_scale[bh * T + j] / v_max);
+        }
+        // masking: causal diagonal block and the ragged last key block
+        const bool masked = (j == nkv_t - 1) && (p.causal || (p.N % kBlockN) != 0);
+        if (masked) {
+          const int limit = (p.causal ? min(row, p.N - 1) : p.N - 1) - j * kBlockN;  // last visible column
 #pragma unroll
-        for (int cb = 0; cb < C::D; cb += 32) {
-          uint32_t ov[32];
-          tmem_ld32(o_tm + cb, ov);
-          tmem_ld_wait<32>(ov);
-          uint32_t packed[16];
+          for (int i = 0; i < 128; ++i)
+            if (i > limit) sr[i] = 0xff800000u;  // -inf
+        }
+        const float m_blk = row_max128(sr) * c;
+        float m_use = m_run;
+        if (m_blk - m_run > C::RESCALE_THRESHOLD) m_use = m_blk;
+        // exponent offset: FP8 folds the V tile scale ratio and a 2^8 pre-scale in
+        const float m_exp = C::FP8 ? (m_use - v_log2_ratio - C::P_PRESCALE_LOG2) : m_use;
+        const bool moved = m_use != m_run;
+        // 2^(m_run - m_use); 0 on the first block
+        const float alpha = moved ? ex2_approx(m_run - m_use) : 1.f;
+        // O_t rescale when this warp moved its maximum (O_t already holds every
+        // earlier P V: the commit behind s_full covers them); it must land
+        // before the first P chunk of this block is released to the MMA.
+        if (j > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
-          if (in_range) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + cb);
+          for (int cb = 0; cb < C::D; cb += 32) {
+            uint32_t ov[32];
+            tmem_ld32(o_tm + cb, ov);
+            tmem_ld_wait<32>(ov);
 #pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            for (int i = 0; i < 32; ++i) ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+            tmem_st32(o_tm + cb, ov);
           }
         }
-        if (p.lse != nullptr && in_range)
-          p.lse[static_cast<size_t>(bh) * p.N + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-      } else {
-        record_timeout();
+        // P_t over the first columns of S_t, chunk by chunk; masked blocks keep
+        // every exponential on MUFU (exact zeros for -inf)
+        uint64_t* pf = p_full + t * C::P_CHUNKS;
+        float sum = masked ? p_row_to_tmem<C, 0u>(sr, c, m_exp, s_tm, pf)
+                           : p_row_to_tmem<C, C::POLY_MASK>(sr, c, m_exp, s_tm, pf);
+        if constexpr (C::FP8) sum *= ex2_approx(-v_log2_ratio - C::P_PRESCALE_LOG2);  // units of 2^m_use
+        l_run = l_run * alpha + sum;
+        m_run = m_use;
       }
+      if (!ok) break;
+      // ---- epilogue: O = O_acc / l, LSE = (m + log2 l) ln 2. The next unit's
+      // first P V (which overwrites O_t) waits for this group's P, which comes
+      // after these TMEM loads.
+      ok = __all_sync(0xffffffffu, waiter.wait(o_done + t, oc & 1));
+      if (!ok) break;
+      ++oc;
+      tc_fence_after();
+      float inv_l = 1.f / l_run;
+      if constexpr (C::FP8) inv_l *= v_max * 0.00390625f;  // undo the V ratio and 2^8 pre-scale
+      const bool in_range = row < p.N;
+      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (in_range ? row : 0)) * C::D;
+#pragma unroll
+      for (int cb = 0; cb < C::D; cb += 32) {
+        uint32_t ov[32];
+        tmem_ld32(o_tm + cb, ov);
+        tmem_ld_wait<32>(ov);
+        uint32_t packed[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          packed[i] = pack_bf16x2(__uint_as_float(ov[2 * i]) * inv_l, __uint_as_float(ov[2 * i + 1]) * inv_l);
+        if (in_range) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + cb);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+      if (p.lse != nullptr && in_range)
+        p.lse[static_cast<size_t>(bh) * p.N + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
+    if (!ok) record_timeout();
   }
 
   // ---- teardown: every TMEM access and MMA of this CTA is complete here
