@@ -93,6 +93,15 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.N = N;
   p.BH = BH;
   p.num_units = BH * npair;
+  // Non-causal: heads per group such that the group's K and V (2 N d bytes per
+  // element per head) take about 48 MB of the 126 MB L2. Causal: all heads.
+  {
+    const long long kv_bytes = 2ll * N * C::D * (C::FP8 ? 1 : 2);
+    long long hg = causal ? BH : (48ll << 20) / (kv_bytes > 0 ? kv_bytes : 1);
+    if (hg < 1) hg = 1;
+    if (hg > BH) hg = BH;
+    p.heads_per_group = static_cast<int>(hg);
+  }
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);

@@ -119,6 +119,7 @@ struct FwdParams {
   int N;          // sequence length
   int BH;         // batch * heads
   int num_units;  // work units = BH * ceil(ceil(N/128) / Q_TILES)
+  int heads_per_group;  // units walk groups of this many heads (K/V of a group fit in L2)
   int causal;
   float scale_log2;       // scale * log2(e)
   __nv_bfloat16* o;       // [BH, N, D]
@@ -215,8 +216,12 @@ __device__ __forceinline__ void p_chunk_bf16(const uint32_t (&sr)[128], int ch, 
   }
 }
 
-// FP8 variant: P = hi + lo with hi = e4m3(p), lo = e4m3(p - hi) (residual in
-// f16); the chunk's 32 keys give 8 hi words and 8 lo words (four codes each).
+// FP8 variant: P = hi + lo, both E4M3: hi = e4m3(p) converted straight from
+// fp32, lo = e4m3(p - hi) with the residual formed in f16x2 (p rounded to f16,
+// hi decoded exactly to f16). The chunk's keys give QUADS hi words and QUADS lo
+// words (four codes each). Conversion forms were chosen by measured contention
+// with MUFU ex2 on B200: e4m3x2 <- f32 +0.2 cycles, f16x2 <- e4m3x2 +0.4,
+// sub.f16x2 +1.2, e4m3x2 <- f16x2 +2.2, f16x2 <- f32 none.
 template <uint32_t POLY_MASK, int QUADS = 8>
 __device__ __forceinline__ void p_chunk_fp8(const uint32_t (&sr)[128], int ch, float c, float m,
                                             uint64_t (&acc)[4], uint32_t (&hi)[QUADS], uint32_t (&lo)[QUADS]) {
@@ -231,12 +236,11 @@ __device__ __forceinline__ void p_chunk_fp8(const uint32_t (&sr)[128], int ch, f
                          p2, p3);
     acc[(2 * i) & 3] = f2_add(acc[(2 * i) & 3], f2_pack(p0, p1));
     acc[(2 * i + 1) & 3] = f2_add(acc[(2 * i + 1) & 3], f2_pack(p2, p3));
-    const uint32_t h01 = pack_f16x2(p0, p1), h23 = pack_f16x2(p2, p3);
-    const uint16_t hi01 = e4m3x2_from_f16x2(h01), hi23 = e4m3x2_from_f16x2(h23);
-    const uint16_t lo01 = e4m3x2_from_f16x2(hsub2_u32(h01, f16x2_from_e4m3x2(hi01)));
-    const uint16_t lo23 = e4m3x2_from_f16x2(hsub2_u32(h23, f16x2_from_e4m3x2(hi23)));
+    const uint16_t hi01 = e4m3x2_from_f32(p0, p1), hi23 = e4m3x2_from_f32(p2, p3);
+    const uint32_t r01 = hsub2_u32(pack_f16x2(p0, p1), f16x2_from_e4m3x2(hi01));
+    const uint32_t r23 = hsub2_u32(pack_f16x2(p2, p3), f16x2_from_e4m3x2(hi23));
     hi[i] = static_cast<uint32_t>(hi01) | (static_cast<uint32_t>(hi23) << 16);
-    lo[i] = static_cast<uint32_t>(lo01) | (static_cast<uint32_t>(lo23) << 16);
+    lo[i] = static_cast<uint32_t>(e4m3x2_from_f16x2(r01)) | (static_cast<uint32_t>(e4m3x2_from_f16x2(r23)) << 16);
   }
 }
 
@@ -295,7 +299,10 @@ __device__ __forceinline__ float p_row_to_tmem(const uint32_t (&sr)[128], float 
 }
 
 // Work unit u of a launch: the pair of Q tiles `qpair` of head `bh`. Units are
-// numbered heaviest causal pairs first (u / BH counts down the pairs). A
+// numbered heaviest causal pairs first (pairs count down; heads vary fastest).
+// Non-causal launches walk the heads in groups whose K and V fit in L2 together,
+// so the CTAs running at the same time share K/V tiles through L2 (causal
+// launches use one group: their balance needs the global heavy-first order). A
 // persistent CTA b takes one unit per round k in snake order: unit
 // k*G + b on even rounds and k*G + G-1-b on odd rounds (G = gridDim.x), so a CTA
 // that got one of the heavier units of a round gets one of the lighter ones in
@@ -311,8 +318,15 @@ struct UnitInfo {
   int qpair, bh, nkv_max;
   int nkv[C::Q_TILES];
   __device__ __forceinline__ UnitInfo(const FwdParams& p, int u, int QB, int NPAIR) {
-    qpair = NPAIR - 1 - u / p.BH;
-    bh = u % p.BH;
+    // heads are taken in groups of heads_per_group (the last group may be
+    // smaller); inside a group, pairs count down and heads vary fastest
+    const int per_group = p.heads_per_group * NPAIR;
+    const int grp = u / per_group;
+    const int h0 = grp * p.heads_per_group;
+    const int hg = min(p.heads_per_group, p.BH - h0);
+    const int v = u - grp * per_group;
+    qpair = NPAIR - 1 - v / hg;
+    bh = h0 + v % hg;
     nkv_max = 0;
 #pragma unroll
     for (int t = 0; t < C::Q_TILES; ++t) {

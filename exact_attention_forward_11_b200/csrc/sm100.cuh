@@ -350,6 +350,12 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+// fp32 pair -> two E4M3 codes (round to nearest even, saturating), element 0 in the low byte
+__device__ __forceinline__ uint16_t e4m3x2_from_f32(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
 // f16x2 -> two E4M3 codes (round to nearest even, saturating), low half -> low byte
 __device__ __forceinline__ uint16_t e4m3x2_from_f16x2(uint32_t h2) {
   uint16_t r;
