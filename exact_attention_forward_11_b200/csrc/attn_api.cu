@@ -182,10 +182,13 @@ attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* s
   if (cudaFuncSetAttribute(attn::fp8_rotate_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            attn::kPrepSmemBytes) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  attn::fp8_rotate_quantize<<<B * H * T, attn::kPrepThreads, attn::kPrepSmemBytes,
+  const int num_tiles = B * H * T;
+  const int sms = sm_count();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  attn::fp8_rotate_quantize<<<num_tiles < sms ? num_tiles : sms, attn::kPrepThreads, attn::kPrepSmemBytes,
                               static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(rot), static_cast<uint8_t*>(x8),
-      scales, N);
+      scales, N, num_tiles);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
