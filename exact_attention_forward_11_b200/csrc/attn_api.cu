@@ -40,15 +40,15 @@ constexpr uint64_t kWaitLimitCycles = 1ull << 31;
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // 3-D map over a contiguous [BH, N, d] tensor: dims {d, N, BH}, box {128 bytes of
-// d, 128 rows, 1}, 128-byte swizzle (the layout the MMA descriptors expect).
+// d, `rows` rows, 1}, 128-byte swizzle (the layout the MMA descriptors expect).
 // Rows past N read as zero.
-bool encode_qkv_map(CUtensorMap* map, const void* base, bool fp8, int d, int N, int BH) {
+bool encode_qkv_map(CUtensorMap* map, const void* base, bool fp8, int d, int N, int BH, int rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return false;
   const int elem = fp8 ? 1 : 2;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * elem, static_cast<cuuint64_t>(N) * d * elem};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), 128u, 1u};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(rows), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                          const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -76,15 +76,16 @@ attn_status check_shape(int B, int H, int N) {
   return ATTN_OK;
 }
 
-template <class C>
+template <int D, bool FP8>
 attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const float* qs,
                        const float* ks, const float* vs, int BH, int N, float scale, int causal,
                        cudaStream_t stream) {
-  CUtensorMap tq, tk, tv;
-  if (!encode_qkv_map(&tq, q, C::FP8, C::D, N, BH) || !encode_qkv_map(&tk, k, C::FP8, C::D, N, BH) ||
-      !encode_qkv_map(&tv, v, C::FP8, C::D, N, BH))
-    return ATTN_ERR_CUDA;
+  using C = attn::FwdCfg<D, FP8>;
   auto kern = attn::attn_fwd_sm100<C>;
+  CUtensorMap tq, tk, tv;
+  if (!encode_qkv_map(&tq, q, FP8, D, N, BH, attn::kBlockM) ||
+      !encode_qkv_map(&tk, k, FP8, D, N, BH, attn::kBlockN) || !encode_qkv_map(&tv, v, FP8, D, N, BH, attn::kBlockN))
+    return ATTN_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int QB = (N + attn::kBlockM - 1) / attn::kBlockM;
@@ -151,8 +152,8 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   if (d == 128)
-    return launch_fwd<attn::FwdCfg<128, false>>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
-  return launch_fwd<attn::FwdCfg<64, false>>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+    return launch_fwd<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+  return launch_fwd<64, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
 }
 
 attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,
@@ -168,8 +169,8 @@ attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const f
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
     return ATTN_ERR_MISALIGNED;
   if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
-  return launch_fwd<attn::FwdCfg<128, true>>(q8, k8, v8, o, lse, q_scale, k_scale, v_scale, B * H, N, scale, causal,
-                                             static_cast<cudaStream_t>(stream));
+  return launch_fwd<128, true>(q8, k8, v8, o, lse, q_scale, k_scale, v_scale, B * H, N, scale, causal,
+                               static_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* scales, int B, int H, int N, int d,

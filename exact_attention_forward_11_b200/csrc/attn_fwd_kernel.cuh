@@ -183,27 +183,30 @@ __device__ __forceinline__ void exp2_pair(float x0, float x1, int i, float& p0, 
   }
 }
 
-// Maximum of 128 values with 3-input max in eight independent chains.
-__device__ __forceinline__ float row_max128(const uint32_t (&sr)[128]) {
+// Maximum of NCOL (64 or 128) values with 3-input max in eight independent chains.
+template <int NCOL = 128>
+__device__ __forceinline__ float row_max(const uint32_t* sr) {
   using b200::max3f;
+  constexpr int L = NCOL / 8;   // values per chain
   float a[8];
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    float m = max3f(__uint_as_float(sr[16 * k]), __uint_as_float(sr[16 * k + 1]), __uint_as_float(sr[16 * k + 2]));
+    float m = max3f(__uint_as_float(sr[L * k]), __uint_as_float(sr[L * k + 1]), __uint_as_float(sr[L * k + 2]));
 #pragma unroll
-    for (int j = 3; j < 15; j += 2)
-      m = max3f(m, __uint_as_float(sr[16 * k + j]), __uint_as_float(sr[16 * k + j + 1]));
-    a[k] = fmaxf(m, __uint_as_float(sr[16 * k + 15]));
+    for (int j = 3; j < L - 1; j += 2)
+      m = max3f(m, __uint_as_float(sr[L * k + j]), __uint_as_float(sr[L * k + j + 1]));
+    a[k] = fmaxf(m, __uint_as_float(sr[L * k + L - 1]));
   }
   return max3f(max3f(a[0], a[1], a[2]), max3f(a[3], a[4], a[5]), fmaxf(a[6], a[7]));
 }
+__device__ __forceinline__ float row_max128(const uint32_t (&sr)[128]) { return row_max<128>(sr); }
 
 // P = 2^(s c - m) for keys [32 ch, 32 ch + 32) of one row, as 16 bf16 pairs in
 // pk; adds the fp32 values to the packed accumulators. The scale-and-subtract
 // is a scalar FMA per element (a packed FMA would compete with MUFU for issue);
 // the sums use packed adds, which do not.
 template <uint32_t POLY_MASK, int PAIRS = 16>
-__device__ __forceinline__ void p_chunk_bf16(const uint32_t (&sr)[128], int ch, float c, float m,
+__device__ __forceinline__ void p_chunk_bf16(const uint32_t* sr, int ch, float c, float m,
                                              uint64_t (&acc)[4], uint32_t (&pk)[PAIRS]) {
   using namespace b200;
 #pragma unroll
@@ -223,7 +226,7 @@ __device__ __forceinline__ void p_chunk_bf16(const uint32_t (&sr)[128], int ch, 
 // with MUFU ex2 on B200: e4m3x2 <- f32 +0.2 cycles, f16x2 <- e4m3x2 +0.4,
 // sub.f16x2 +1.2, e4m3x2 <- f16x2 +2.2, f16x2 <- f32 none.
 template <uint32_t POLY_MASK, int QUADS = 8>
-__device__ __forceinline__ void p_chunk_fp8(const uint32_t (&sr)[128], int ch, float c, float m,
+__device__ __forceinline__ void p_chunk_fp8(const uint32_t* sr, int ch, float c, float m,
                                             uint64_t (&acc)[4], uint32_t (&hi)[QUADS], uint32_t (&lo)[QUADS]) {
   using namespace b200;
 #pragma unroll
@@ -454,15 +457,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
   } else if (warp == C::MMA_WARP) {
     // ======================= MMA issuer =======================
-    // Warp-uniform loop; one elected lane issues every tcgen05.mma and commit.
+    // Warp-uniform loop. One lane, elected once, issues every tcgen05.mma and
+    // commit (a commit tracks the MMAs of its own thread only); the instructions
+    // are predicated on it, so the warp never diverges. The issue rate of this
+    // warp, not the tensor pipe, bounds the MMA segments: under the softmax
+    // load on its SM sub-partition one MMA takes ~65-80 cycles to issue.
     regs_decrease<C::REGS_CONTROL>();
     auto wait_all = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, waiter.wait(bar, parity));
     };
-    auto commit = [&](uint64_t* bar) {
-      if (elect_one()) mma_commit(bar);
-      __syncwarp();
-    };
+    const uint32_t leader = elect_one() ? 1u : 0u;
+    auto commit = [&](uint64_t* bar) { mma_commit(bar, leader); };
     constexpr uint32_t fmt = C::FP8 ? 0u : 1u;
     constexpr uint32_t idesc_s = instr_desc(fmt, 128, kBlockN, 0, 0);
     constexpr uint32_t idesc_o = instr_desc(fmt, 128, C::D, 0, 1);
@@ -484,13 +489,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const uint32_t off = ((kk / per_chunk) * C::CHUNK_BYTES + (kk % per_chunk) * 32) >> 4;
         const uint64_t da = smem_desc(qa + off, hi_kmaj);
         const uint64_t db = smem_desc(ka + off, hi_kmaj);
-        if (elect_one()) {
-          if constexpr (C::FP8)
-            mma_f8_ss(d_tmem, da, db, idesc_s, kk > 0);
-          else
-            mma_f16_ss(d_tmem, da, db, idesc_s, kk > 0);
-        }
-        __syncwarp();
+        if constexpr (C::FP8)
+          mma_f8_ss(d_tmem, da, db, idesc_s, kk > 0, leader);
+        else
+          mma_f16_ss(d_tmem, da, db, idesc_s, kk > 0, leader);
       }
     };
     // O_t (+)= P_t V_j for the keys of P chunk c: P from TMEM (over S_t), V
@@ -509,13 +511,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const int kk = term * C::PV_KSTEPS + kv;          // K step within [hi | lo]
           const uint64_t db = smem_desc(va + ((kv * C::UMMA_K * 128) >> 4), hi_mnmaj);
           const uint32_t accum = (acc || term > 0 || i > 0) ? 1u : 0u;
-          if (elect_one()) {
-            if constexpr (C::FP8)
-              mma_f8_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum);
-            else
-              mma_f16_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum);
-          }
-          __syncwarp();
+          if constexpr (C::FP8)
+            mma_f8_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum, leader);
+          else
+            mma_f16_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum, leader);
         }
     };
     uint32_t g = 0;                       // K/V tiles consumed so far (same count as the producer's)
