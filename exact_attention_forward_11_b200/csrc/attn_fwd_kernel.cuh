@@ -76,7 +76,10 @@ struct FwdCfg {
   static constexpr int PV_KSTEPS_TOTAL = FP8 ? 2 * PV_KSTEPS : PV_KSTEPS;
   // P is handed to the MMA in P_CHUNKS chunks of 64 keys, each with its own
   // barrier, so P V of a tile starts under the tile's remaining exponentials.
-  static constexpr int P_CHUNKS = 2;
+#ifndef ATTN_P_CHUNKS
+#define ATTN_P_CHUNKS 2
+#endif
+  static constexpr int P_CHUNKS = ATTN_P_CHUNKS;
   static constexpr int KEYS_PER_CHUNK = kBlockN / P_CHUNKS;
   static constexpr int NUM_SOFTMAX_THREADS = 128 * Q_TILES;
   static constexpr int PRODUCER_WARP = NUM_SOFTMAX_THREADS / 32;
