@@ -160,6 +160,15 @@ def gpu_smi_id(dev, local):
     return vis.split(",")[local] if vis else str(local)
 
 
+def sustained_bf16_peak():
+    """The measured bf16 GEMM rate over seconds under the power cap (None if absent)."""
+    path = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f).get("bf16_tflops_sustained")
+    return None
+
+
 def measured_peaks():
     path = os.path.join(HERE, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -314,6 +323,13 @@ def run_ours(args):
             "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(args.workload),
             "peak_source": f"{peak_src} bf16 burst" + (" x2 (fp8 nominal ratio)" if w.fp8 else ""),
             "kernel": "attn_fwd_sm100" + ("+fp8_rotate_quantize" if w.fp8 else "")}
+    sus = sustained_bf16_peak()
+    if sus:
+        # the timed loop runs long enough to meet the 1 kW power cap (see "clocks"); the
+        # sustained GEMM rate is the same-conditions denominator
+        sus = sus * 2 if w.fp8 else sus
+        roof["frac_of_sustained_peak"] = round(achieved / sus, 4)
+        roof["sustained_peak"] = sus
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_baseline(w, budget_s=float(os.environ.get("ATTN_CPU_BASELINE_S", "15")))
