@@ -29,6 +29,7 @@ SIGNATURES = {
     "attn_quantize_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "attn_get_device_status": (_I, [_P]),
+    "attn_fwd_inject_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, ctypes.c_ulonglong, _P]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_abi_version": (_I, []),
 }
@@ -66,6 +67,12 @@ def attn_quantize_fp8(x, rot, x8, scales, B, H, N, d, stream):
 
 def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, scale, causal, stream):
     return load().attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, scale, causal, stream)
+
+
+def attn_fwd_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit, wait_limit_cycles, stream):
+    """Testing hook (include/attn_b200_testing.h): attn_fwd with one K tile withheld."""
+    return load().attn_fwd_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit,
+                                          wait_limit_cycles, stream)
 
 
 def attn_get_device_status(stream):

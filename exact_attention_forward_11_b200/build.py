@@ -35,7 +35,7 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "attn_b200.h"), __file__]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, h) for h in os.listdir(INCLUDE)] + [__file__]
     return any(os.path.getmtime(p) > t for p in deps)
 
 

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "attn_b200.h"
+#include "attn_b200_testing.h"
 #include "attn_fwd_kernel.cuh"
 #include "fp8_prep_kernel.cuh"
 
@@ -79,7 +80,7 @@ attn_status check_shape(int B, int H, int N) {
 template <int D, bool FP8>
 attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const float* qs,
                        const float* ks, const float* vs, int BH, int N, float scale, int causal,
-                       cudaStream_t stream) {
+                       cudaStream_t stream, int fault_unit = -1, uint64_t wait_limit = kWaitLimitCycles) {
   using C = attn::FwdCfg<D, FP8>;
   auto kern = attn::attn_fwd_sm100<C>;
   CUtensorMap tq, tk, tv;
@@ -110,7 +111,8 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.q_scale = qs;
   p.k_scale = ks;
   p.v_scale = vs;
-  p.timeout_cycles = kWaitLimitCycles;
+  p.timeout_cycles = wait_limit;
+  p.fault_unit = fault_unit;
   // persistent grid: one CTA per SM (shared memory and TMEM allow one), each
   // walking the units blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
@@ -154,6 +156,22 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   if (d == 128)
     return launch_fwd<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
   return launch_fwd<64, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+}
+
+attn_status attn_fwd_inject_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                    int N, int d, float scale, int causal, int fault_unit,
+                                    unsigned long long wait_limit_cycles, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (fault_unit < 0 || wait_limit_cycles < 1024) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
+    return ATTN_ERR_MISALIGNED;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
+  return launch_fwd<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, B * H, N, scale, causal,
+                                static_cast<cudaStream_t>(stream), fault_unit, wait_limit_cycles);
 }
 
 attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,

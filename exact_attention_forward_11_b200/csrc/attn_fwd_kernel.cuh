@@ -131,6 +131,7 @@ struct FwdParams {
   const float* k_scale;
   const float* v_scale;
   uint64_t timeout_cycles;  // per pipeline wait, in SM cycles
+  int fault_unit;           // testing only: the producer withholds this unit's first K tile (-1: none)
 };
 
 // Bounded wait that ignores the abort word (used only while draining after an
@@ -436,6 +437,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       __syncwarp();
       ++q_loads;
       for (int i = 0; i < 2 * w.nkv_max; ++i, ++g) {
+        // testing hook: a tile that is never loaded leaves its full barrier
+        // incomplete, so the MMA warp's bounded wait runs out
+        if (i == 0 && u == p.fault_unit) continue;
         const uint32_t slot = g % C::NSLOT;
         if (g >= C::NSLOT && !(ok = wait_all(kv_empty + slot, ((g / C::NSLOT) - 1) & 1))) break;
         const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;

@@ -1,0 +1,42 @@
+/*
+ * attn_b200_testing.h - testing hook of the attention library (not part of the
+ * operation; the pages define no counterpart).
+ *
+ * attn_fwd_inject_timeout - attn_fwd for BF16, d = 128, with one failure
+ * planted on purpose so that the bounded-wait path of the kernel can be run on
+ * a GPU without faulting it: the TMA producer of the CTA that processes work
+ * unit `fault_unit` never loads that unit's first K tile, so the mbarrier the
+ * MMA warp waits on is never completed. Every pipeline wait of the launch
+ * gives up after `wait_limit_cycles` SM cycles (instead of the 2^31 that
+ * attn_fwd uses); the CTA then sets its abort word, lets its in-flight copies
+ * and MMAs land, releases its tensor memory and exits, and the launch records
+ * ATTN_ERR_TIMEOUT in the device status word (read and cleared by
+ * attn_get_device_status). Other CTAs are not affected; the CUDA context stays
+ * usable, and the output of the failed unit is undefined.
+ *
+ * Work units are numbered as the kernel walks them: unit u covers one head and
+ * two consecutive 128-row Q tiles (u < B*H*ceil(ceil(N/128)/2)).
+ *
+ * Arguments as for attn_fwd (device pointers, [B, H, N, 128] bf16, 16-byte
+ * aligned), plus fault_unit >= 0 and wait_limit_cycles >= 1024.
+ * Returns the launch status (ATTN_OK when the kernel was launched) or the same
+ * host-side argument errors as attn_fwd; ATTN_ERR_UNSUPPORTED unless d == 128.
+ */
+#ifndef ATTN_B200_TESTING_H
+#define ATTN_B200_TESTING_H
+
+#include "attn_b200.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+ATTN_API attn_status attn_fwd_inject_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
+                                             int B, int H, int N, int d, float scale, int causal, int fault_unit,
+                                             unsigned long long wait_limit_cycles, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_B200_TESTING_H */

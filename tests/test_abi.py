@@ -1,6 +1,7 @@
 """The C-ABI library loads, exports every symbol include/attn_b200.h declares, and
 rejects bad arguments on the host before any CUDA call (so this runs without a GPU)."""
 import ctypes
+import glob
 import os
 import re
 import subprocess
@@ -9,10 +10,11 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "attn_b200.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def declared_symbols():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)))
 
 
