@@ -18,7 +18,8 @@
 // per CTA as fp32. Thread (ty, tx) = (tid % 16, tid / 16) owns the outputs of
 // rows ty + 16 i (i < 8) and columns 8 tx .. 8 tx + 7: interleaved rows make the
 // float4 reads of x from shared memory conflict-free, and the k loop runs four
-// steps per round of loads while every output still accumulates in k order.
+// steps per round of loads while every output still accumulates in k order
+// (two columns per packed fma.rn.f32x2).
 // Rows past N read as zero and are not written.
 #pragma once
 
@@ -84,10 +85,14 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 
     float acc[8][8];
     if (rotate) {
+      // packed FMAs on column pairs: fma.rn.f32x2 rounds each lane exactly like a
+      // scalar fma.rn, so every output still accumulates in k order, once-rounded
+      // per step (bit-identical), at half the instruction count
+      uint64_t acc2[8][4];
 #pragma unroll
       for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+        for (int j = 0; j < 4; ++j) acc2[i][j] = 0ull;
 #pragma unroll 1
       for (int k0 = 0; k0 < kPrepTile; k0 += 4) {
         float4 xa[8];
@@ -97,15 +102,21 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         for (int kk = 0; kk < 4; ++kk) {
           const float4 r0 = *reinterpret_cast<const float4*>(rs + (k0 + kk) * kPrepLd + tx * 8);
           const float4 r1 = *reinterpret_cast<const float4*>(rs + (k0 + kk) * kPrepLd + tx * 8 + 4);
-          const float b[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
+          const uint64_t b2[4] = {b200::f2_pack(r0.x, r0.y), b200::f2_pack(r0.z, r0.w), b200::f2_pack(r1.x, r1.y),
+                                  b200::f2_pack(r1.z, r1.w)};
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
             const float a = kk == 0 ? xa[i].x : kk == 1 ? xa[i].y : kk == 2 ? xa[i].z : xa[i].w;
+            const uint64_t a2 = b200::f2_pack(a, a);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[i][j] = __fmaf_rn(a, b[j], acc[i][j]);
+            for (int j = 0; j < 4; ++j) acc2[i][j] = b200::f2_fma(a2, b2[j], acc2[i][j]);
           }
         }
       }
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) b200::f2_unpack(acc2[i][j], acc[i][2 * j], acc[i][2 * j + 1]);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
