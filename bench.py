@@ -92,7 +92,10 @@ def shard_seed(w, rank):
 
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
-    """Samples SM clock, power and throttle reasons with nvidia-smi while running."""
+    """Samples SM clock, power and throttle reasons with nvidia-smi every 50 ms.
+    Sampling is running before the timed region starts (entry waits for the first
+    sample), every sample is timestamped, and the summary keeps the samples taken
+    between mark_start() and mark_end() (all samples if none fall inside)."""
     FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
               "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
               "clocks_event_reasons.sw_power_cap"]
@@ -100,7 +103,8 @@ class ClockSampler:
     def __init__(self, gpu_id):
         self.gpu_id = gpu_id
         self.proc = None
-        self.lines = []
+        self.lines = []          # (host time, csv line)
+        self.window = None
 
     def __enter__(self):
         try:
@@ -110,14 +114,23 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
-            time.sleep(0.15)
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 10.0 and self.proc.poll() is None:
+                time.sleep(0.02)
         except OSError:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark_start(self):
+        self.window = [time.time(), None]
+
+    def mark_end(self):
+        if self.window is not None:
+            self.window[1] = time.time()
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -132,7 +145,11 @@ class ClockSampler:
         import statistics
         sms, maxs, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        lines = self.lines
+        if self.window is not None and self.window[1] is not None:
+            inside = [x for x in lines if self.window[0] <= x[0] <= self.window[1]]
+            lines = inside if inside else lines
+        for _, ln in lines:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) != len(self.FIELDS):
                 continue
@@ -147,7 +164,7 @@ class ClockSampler:
         if not sms:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
-                "samples": len(sms)}
+                "samples": len(sms), "timed_window_only": lines is not self.lines}
 
 
 def gpu_smi_id(dev, local):
@@ -217,7 +234,7 @@ class Step:
             raise lib.AttnError(st, "attn_fwd_fp8")
 
 
-def time_device(step, stream, steps, warmup, world, dev):
+def time_device(step, stream, steps, warmup, world, dev, clk=None):
     import torch
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -226,11 +243,15 @@ def time_device(step, stream, steps, warmup, world, dev):
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if clk is not None:
+        clk.mark_start()
     e0.record(stream)
     for _ in range(steps):
         step.run_device(stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
+    if clk is not None:
+        clk.mark_end()
     barrier(world, dev)
     return e0.elapsed_time(e1)  # ms for `steps` steps, this rank
 
@@ -298,7 +319,7 @@ def run_ours(args):
     stream = torch.cuda.Stream(dev)
     step = Step(lib, w, x, dev)
     with ClockSampler(gpu_smi_id(dev, local)) as clk:
-        ms_rank = time_device(step, stream, args.steps, max(3, args.warmup), world, dev)
+        ms_rank = time_device(step, stream, args.steps, max(3, args.warmup), world, dev, clk)
     st = lib.attn_get_device_status(stream.cuda_stream)
     if st != lib.ATTN_OK:
         raise lib.AttnError(st, "device status")
