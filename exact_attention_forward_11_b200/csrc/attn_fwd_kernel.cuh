@@ -94,8 +94,12 @@ struct FwdCfg {
   static constexpr uint32_t O_COL0 = 256;
   // Lazy rescaling: the running maximum is only moved when a new block raises it
   // by more than this (log2 units). Exact for any value; 8 keeps bf16 P <= 256.
-  // FP8 P must stay below 448 after a 2^8 pre-scale, so it moves every time.
-  static constexpr float RESCALE_THRESHOLD = FP8 ? 0.0f : 8.0f;
+  // FP8 P must stay at or below 448 (the largest E4M3 value) after a 2^8
+  // pre-scale: a lag of at most 0.8 keeps it <= 2^8.8 = 445.7.
+#ifndef ATTN_FP8_RESCALE_THRESHOLD
+#define ATTN_FP8_RESCALE_THRESHOLD 0.8f
+#endif
+  static constexpr float RESCALE_THRESHOLD = FP8 ? ATTN_FP8_RESCALE_THRESHOLD : 8.0f;
   static constexpr float P_PRESCALE_LOG2 = 8.0f;  // FP8 only
   // Pairs of P values (by index mod 8) whose exp2 runs as a polynomial on the
   // FMA pipe instead of the MUFU unit, in blocks that need no masking. MUFU
