@@ -109,19 +109,31 @@ def _shape4(q):
     return tuple(q.shape)
 
 
+def _expect(t, name, shape, dtype, device):
+    """Every tensor handed to the library must be a contiguous CUDA tensor of the
+    exact shape and dtype, on the same device as the first input (the kernels
+    read and write through raw device pointers)."""
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+
+
 def forward(q, k, v, causal=False, scale=None, out=None, lse=None, with_lse=True, stream=None):
     """O, LSE = attention(q, k, v) for bf16 CUDA tensors [B, H, N, d]."""
     import torch
     B, H, N, d = _shape4(q)
-    for t in (k, v):
-        if tuple(t.shape) != (B, H, N, d) or t.dtype != torch.bfloat16 or not t.is_contiguous():
-            raise ValueError("k, v must match q")
-    if q.dtype != torch.bfloat16:
-        raise ValueError("q must be bf16")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _expect(t, name, (B, H, N, d), torch.bfloat16, q.device)
     if out is None:
         out = torch.empty_like(q)
+    _expect(out, "out", (B, H, N, d), torch.bfloat16, q.device)
     if lse is None and with_lse:
         lse = torch.empty((B, H, N), device=q.device, dtype=torch.float32)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, N), torch.float32, q.device)
     sc = 0.0 if scale is None else float(scale)
     _check(attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc,
                     int(bool(causal)), ATTN_BF16, _stream_ptr(q, stream)), "attn_fwd")
@@ -132,6 +144,9 @@ def quantize_fp8(x, rot=None, stream=None):
     """(codes uint8 [B,H,N,d], scales fp32 [B,H,ceil(N/128)]) of a bf16 tensor."""
     import torch
     B, H, N, d = _shape4(x)
+    _expect(x, "x", (B, H, N, d), torch.bfloat16, x.device)
+    if rot is not None:
+        _expect(rot, "rot", (d, d), torch.bfloat16, x.device)
     x8 = torch.empty((B, H, N, d), device=x.device, dtype=torch.uint8)
     scales = torch.empty((B, H, (N + TILE - 1) // TILE), device=x.device, dtype=torch.float32)
     _check(attn_quantize_fp8(x.data_ptr(), _ptr(rot), x8.data_ptr(), scales.data_ptr(), B, H, N, d,
@@ -144,10 +159,18 @@ def forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale=None,
     """O (bf16), LSE from E4M3 codes and their per-tile scales."""
     import torch
     B, H, N, d = _shape4(q8)
+    T = (N + TILE - 1) // TILE
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _expect(t, name, (B, H, N, d), torch.uint8, q8.device)
+    for name, t in (("q_scale", q_scale), ("k_scale", k_scale), ("v_scale", v_scale)):
+        _expect(t, name, (B, H, T), torch.float32, q8.device)
     if out is None:
         out = torch.empty((B, H, N, d), device=q8.device, dtype=torch.bfloat16)
+    _expect(out, "out", (B, H, N, d), torch.bfloat16, q8.device)
     if lse is None and with_lse:
         lse = torch.empty((B, H, N), device=q8.device, dtype=torch.float32)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, N), torch.float32, q8.device)
     sc = 0.0 if scale is None else float(scale)
     _check(attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_scale.data_ptr(), k_scale.data_ptr(),
                         v_scale.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc, int(bool(causal)),
