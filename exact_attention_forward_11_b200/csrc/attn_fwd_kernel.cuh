@@ -27,8 +27,10 @@
 //                                        E4M3 quads) is written over its first
 //                                        columns once S_t has been read
 //   O_t  columns [256 + D t, 256 + D t + D)   fp32 output accumulator of tile t
-// Shared memory: Q tiles (resident for the CTA) + a ring of NSLOT tile slots
-// that the producer fills in the order K_0, V_0, K_1, V_1, ...
+// Shared memory: the Q tiles of the current work unit (reloaded for the next unit
+// once its last S MMAs have completed) + a ring of NSLOT tile slots that the
+// producer fills in the order K_0, V_0, K_1, V_1, ... CTAs are persistent (one
+// per SM) and walk the work units of the launch (see unit_of_round).
 //
 // Per KV block j the MMA thread issues, for t = 0, 1:
 //   O_t (+)= P_t(j-1) V_{j-1}   then   S_t = Q_t K_j^T
