@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -70,6 +71,31 @@ int sm_count() {
   return n;
 }
 
+// Raises a kernel's dynamic shared-memory limit once per device (the attribute
+// belongs to the function on the current device; later calls skip the driver
+// call). `tag` identifies the kernel. A failed launch forgets the flag, so a
+// context that was reset gets the attribute again on the next call.
+std::atomic<uint32_t> g_smem_done[64][8];
+
+void forget_smem(int tag) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && tag < 8)
+    g_smem_done[dev][tag].store(0u, std::memory_order_release);
+}
+
+bool set_smem_once(const void* func, int bytes, int tag) {
+  auto& done = g_smem_done;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
+  if (dev < 64 && tag < 8 && done[dev][tag].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+  if (dev < 64 && tag < 8) done[dev][tag].store(1u, std::memory_order_release);
+  return true;
+}
+
+template <int D, bool FP8>
+constexpr int fwd_tag() { return FP8 ? 2 : (D == 128 ? 0 : 1); }
+
 attn_status check_shape(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
   const long long rows = static_cast<long long>(B) * H * N;
@@ -87,8 +113,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   if (!encode_qkv_map(&tq, q, FP8, D, N, BH, attn::kBlockM) ||
       !encode_qkv_map(&tk, k, FP8, D, N, BH, attn::kBlockN) || !encode_qkv_map(&tv, v, FP8, D, N, BH, attn::kBlockN))
     return ATTN_ERR_CUDA;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
-    return ATTN_ERR_CUDA;
+  if (!set_smem_once(reinterpret_cast<const void*>(kern), C::SMEM_BYTES, fwd_tag<D, FP8>())) return ATTN_ERR_CUDA;
   const int QB = (N + attn::kBlockM - 1) / attn::kBlockM;
   const int npair = (QB + C::Q_TILES - 1) / C::Q_TILES;
   attn::FwdParams p;
@@ -119,7 +144,11 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   if (sms <= 0) return ATTN_ERR_CUDA;
   const int grid = p.num_units < sms ? p.num_units : sms;
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) {
+    forget_smem(fwd_tag<D, FP8>());
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 }  // namespace
@@ -198,8 +227,7 @@ attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* s
   if (d != attn::kPrepTile) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(x8) || (rot != nullptr && !aligned16(rot))) return ATTN_ERR_MISALIGNED;
   const int T = (N + attn::kPrepTile - 1) / attn::kPrepTile;
-  if (cudaFuncSetAttribute(attn::fp8_rotate_quantize, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           attn::kPrepSmemBytes) != cudaSuccess)
+  if (!set_smem_once(reinterpret_cast<const void*>(attn::fp8_rotate_quantize), attn::kPrepSmemBytes, 3))
     return ATTN_ERR_CUDA;
   const int num_tiles = B * H * T;
   const int sms = sm_count();
@@ -208,7 +236,11 @@ attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* s
                               static_cast<cudaStream_t>(stream)>>>(
       static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(rot), static_cast<uint8_t*>(x8),
       scales, N, num_tiles);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+  if (cudaGetLastError() != cudaSuccess) {
+    forget_smem(3);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 attn_status attn_get_device_status(void* stream) {
