@@ -91,39 +91,101 @@ def shard_seed(w, rank):
 
 
 # ------------------------------------------------------------------ clocks
+REASON_NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+
+
 class ClockSampler:
-    """Samples SM clock, power and throttle reasons with nvidia-smi every 50 ms.
-    Sampling is running before the timed region starts (entry waits for the first
-    sample), every sample is timestamped, and the summary keeps the samples taken
-    between mark_start() and mark_end() (all samples if none fall inside)."""
-    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
-              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
-              "clocks_event_reasons.sw_power_cap"]
+    """Samples the SM clock, its maximum and the throttle reasons while the timed
+    region runs. NVML is read directly every ~2 ms (read-only queries), so even a
+    timed region of ~10 ms holds several samples; without NVML, nvidia-smi is
+    polled every 50 ms instead. Sampling is running before the timed region
+    starts (entry waits for the first sample), every sample carries its host
+    time, and the summary keeps the samples taken between mark_start() and
+    mark_end() (all samples if none fall inside).
 
-    def __init__(self, gpu_id):
+    A sample is (host time, sm MHz, max sm MHz, set of active reason names)."""
+    SMI_FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+                  "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+                  "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_id, period_s=0.002):
         self.gpu_id = gpu_id
-        self.proc = None
-        self.lines = []          # (host time, csv line)
+        self.period_s = period_s
+        self.samples = []
         self.window = None
+        self.source = None
+        self._stop = threading.Event()
+        self.proc = None
+        self.thread = None
 
-    def __enter__(self):
+    # ---- NVML
+    def _nvml_loop(self, pynvml, h):
+        bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+            except pynvml.NVMLError:
+                break
+            self.samples.append((time.time(), float(sm), float(mx), {n for n, b in bits.items() if r & b}))
+            time.sleep(self.period_s)
+
+    def _start_nvml(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            gid = str(self.gpu_id)
+            h = (pynvml.nvmlDeviceGetHandleByUUID(gid) if gid.startswith("GPU-")
+                 else pynvml.nvmlDeviceGetHandleByIndex(int(gid)))
+        except Exception:
+            return False
+        self.source = "nvml"
+        self.thread = threading.Thread(target=self._nvml_loop, args=(pynvml, h), daemon=True)
+        self.thread.start()
+        return True
+
+    # ---- nvidia-smi fallback
+    def _smi_read(self):
+        for line in self.proc.stdout:
+            smp = self.parse_smi_line(time.time(), line)
+            if smp is not None:
+                self.samples.append(smp)
+
+    @classmethod
+    def parse_smi_line(cls, t, line):
+        parts = [p.strip() for p in line.strip().split(",")]
+        if len(parts) != len(cls.SMI_FIELDS):
+            return None
+        try:
+            sm, mx = float(parts[0]), float(parts[1])
+        except ValueError:
+            return None
+        return (t, sm, mx, {n for n, v in zip(REASON_NAMES, parts[3:]) if v.lower() == "active"})
+
+    def _start_smi(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu_id), "--query-gpu=" + ",".join(self.FIELDS),
+                ["nvidia-smi", "-i", str(self.gpu_id), "--query-gpu=" + ",".join(self.SMI_FIELDS),
                  "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-            t0 = time.time()
-            while not self.lines and time.time() - t0 < 10.0 and self.proc.poll() is None:
-                time.sleep(0.02)
         except OSError:
             self.proc = None
-        return self
+            return False
+        self.source = "nvidia-smi"
+        self.thread = threading.Thread(target=self._smi_read, daemon=True)
+        self.thread.start()
+        return True
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+    def __enter__(self):
+        if self._start_nvml() or self._start_smi():
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 10.0:
+                time.sleep(0.005)
+        return self
 
     def mark_start(self):
         self.window = [time.time(), None]
@@ -133,38 +195,33 @@ class ClockSampler:
             self.window[1] = time.time()
 
     def __exit__(self, *exc):
+        time.sleep(0.01)
+        self._stop.set()
         if self.proc is not None:
-            time.sleep(0.1)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
         import statistics
-        sms, maxs, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        lines = self.lines
+        samples = list(self.samples)
+        inside = samples
         if self.window is not None and self.window[1] is not None:
-            inside = [x for x in lines if self.window[0] <= x[0] <= self.window[1]]
-            lines = inside if inside else lines
-        for _, ln in lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
-            try:
-                sms.append(float(parts[0]))
-                maxs.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[3:]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sms:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs), "reasons": sorted(reasons),
-                "samples": len(sms), "timed_window_only": lines is not self.lines}
+            inside = [x for x in samples if self.window[0] <= x[0] <= self.window[1]]
+        window_only = bool(inside) and self.window is not None and self.window[1] is not None
+        use = inside if inside else samples
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "source": self.source}
+        reasons = set()
+        for x in use:
+            reasons |= x[3]
+        return {"sm_mhz": statistics.median(x[1] for x in use), "sm_max_mhz": max(x[2] for x in use),
+                "reasons": sorted(reasons), "samples": len(use), "timed_window_only": window_only,
+                "source": self.source}
 
 
 def gpu_smi_id(dev, local):
@@ -228,10 +285,15 @@ class Step:
             self.codes = [torch.empty((w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8) for _ in range(3)]
             self.scales = [torch.empty((w.B, w.H, T), device=dev, dtype=torch.float32) for _ in range(3)]
         self.launches = 4 if w.fp8 else 1
+        self.kernels = (["fp8_rotate_quantize", "fp8_quantize", "attn_fwd_sm100"] if w.fp8
+                        else ["attn_fwd_sm100"])
 
-    def run_device(self, stream):
+    def run_device(self, stream, mark=None):
+        """Launches one step on `stream`; mark(kernel name), if given, is called
+        after each launch (the timed loop records a CUDA event there)."""
         lib, w = self.lib, self.w
         s = stream.cuda_stream
+        mark = mark or (lambda name: None)
         if not w.fp8:
             q, k, v, o, lse = self.sets[self.i]
             self.i = (self.i + 1) % self.copies
@@ -239,20 +301,26 @@ class Step:
                               w.B, w.H, w.N, w.d, w.scale, int(w.causal), lib.ATTN_BF16, s)
             if st:
                 raise lib.AttnError(st, "attn_fwd")
+            mark("attn_fwd_sm100")
             return
         for src, rot, c8, sc in zip((self.q, self.k, self.v), (self.rot, self.rot, None), self.codes, self.scales):
             st = lib.attn_quantize_fp8(src.data_ptr(), None if rot is None else rot.data_ptr(), c8.data_ptr(),
                                        sc.data_ptr(), w.B, w.H, w.N, w.d, s)
             if st:
                 raise lib.AttnError(st, "attn_quantize_fp8")
+            mark("fp8_rotate_quantize" if rot is not None else "fp8_quantize")
         st = lib.attn_fwd_fp8(*(c.data_ptr() for c in self.codes), *(c.data_ptr() for c in self.scales),
                               self.o.data_ptr(), self.lse.data_ptr(), w.B, w.H, w.N, w.d, w.scale,
                               int(w.causal), s)
         if st:
             raise lib.AttnError(st, "attn_fwd_fp8")
+        mark("attn_fwd_sm100")
 
 
 def time_device(step, stream, steps, warmup, world, dev, clk=None):
+    """Returns (ms for `steps` steps on this rank, {kernel: mean ms per launch}).
+    Events are recorded on the launching stream before the loop and after every
+    launch, so each kernel's time is the gap between its neighbouring events."""
     import torch
     with torch.cuda.stream(stream):
         for _ in range(warmup):
@@ -261,17 +329,35 @@ def time_device(step, stream, steps, warmup, world, dev, clk=None):
     barrier(world, dev)
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    marks = []
+
+    def mark(name):
+        ev = torch.cuda.Event(enable_timing=True)
+        ev.record(stream)
+        marks.append((name, ev))
+
+    # a one-launch step needs no events between launches: its kernel time is the step time
+    many = step.launches > 1
     if clk is not None:
         clk.mark_start()
     e0.record(stream)
     for _ in range(steps):
-        step.run_device(stream)
+        step.run_device(stream, mark if many else None)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     if clk is not None:
         clk.mark_end()
     barrier(world, dev)
-    return e0.elapsed_time(e1)  # ms for `steps` steps, this rank
+    total = e0.elapsed_time(e1)
+    if not many:
+        return total, {step.kernels[0]: total / steps}
+    per = {}
+    prev = e0
+    for name, ev in marks:
+        per.setdefault(name, []).append(prev.elapsed_time(ev))
+        prev = ev
+    return total, {k: sum(v) / len(v) for k, v in per.items()}
+
 
 
 def time_e2e(lib, w, x, dev, stream, steps):
@@ -316,6 +402,90 @@ def time_e2e(lib, w, x, dev, stream, steps):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
+SMS = 148
+# dense tensor-core FLOPs per SM per clock (a 128x128x16 bf16 MMA step in 64 cycles;
+# E4M3 at twice that rate) and NVIDIA's datasheet dense peaks
+FLOP_PER_CLK_SM = {"bf16": 8192, "fp8": 16384}
+DATASHEET_TFLOPS = {"bf16": 2250.0, "fp8": 4500.0}
+
+
+def hw_peak_tflops(dt, sm_mhz):
+    """Dense tensor-core peak of all SMs at the sampled SM clock."""
+    return None if sm_mhz is None else SMS * FLOP_PER_CLK_SM[dt] * sm_mhz * 1e6 / 1e12
+
+
+def prep_bytes(w):
+    """Algorithmic bytes of one FP8 preparation launch: bf16 read, one code byte
+    written per element, one fp32 scale per 128-token tile."""
+    T = (w.N + 127) // 128
+    return w.B * w.H * w.N * w.d * 3 + 4 * w.B * w.H * T
+
+
+def roofline(w, kern_ms, sm_mhz, workload):
+    """Roofline object of the dominant kernel (the attention kernel), from its
+    mean launch time measured with CUDA events in the timed loop."""
+    peak_bf16, hbm, peak_src = measured_peaks()
+    dt = "fp8" if w.fp8 else "bf16"
+    k_ms = kern_ms["attn_fwd_sm100"]
+    if w.N < 1024 and not w.fp8:
+        # small N (ViT shapes): arithmetic intensity below the ridge point, so the
+        # roofline is HBM: algorithmic bytes = Q, K, V read once + O written (bf16) + LSE (fp32)
+        bytes_launch = 2 * w.B * w.H * w.N * w.d * 4 + 4 * w.B * w.H * w.N
+        gbs = bytes_launch / (k_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(gbs / hbm, 4), "traffic": traffic_per_launch(workload),
+                "peak_source": f"{peak_src} copy bandwidth", "kernel": "attn_fwd_sm100",
+                "algorithmic_bytes": bytes_launch, "kernel_ms": round(k_ms, 5)}
+    achieved = w.flops / (k_ms * 1e-3) / 1e12
+    peak = peak_bf16 * (2 if w.fp8 else 1)
+    roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(workload),
+            "peak_source": f"{peak_src} bf16 burst" + (" x2 (fp8 nominal ratio)" if w.fp8 else ""),
+            "kernel": "attn_fwd_sm100", "algorithmic_flops": w.flops, "kernel_ms": round(k_ms, 5),
+            "datasheet_peak": DATASHEET_TFLOPS[dt],
+            "frac_of_datasheet_peak": round(achieved / DATASHEET_TFLOPS[dt], 4)}
+    hw = hw_peak_tflops(dt, sm_mhz)
+    if hw:
+        roof["hw_peak_at_sampled_clock"] = round(hw, 1)
+        roof["frac_of_hw_peak_at_sampled_clock"] = round(achieved / hw, 4)
+    sus = sustained_bf16_peak()
+    if sus:
+        # a long timed loop meets the 1 kW power cap (see "clocks"); the sustained
+        # GEMM rate is the same-conditions denominator
+        sus = sus * 2 if w.fp8 else sus
+        roof["frac_of_sustained_peak"] = round(achieved / sus, 4)
+        roof["sustained_peak"] = sus
+    if w.fp8:
+        pb = prep_bytes(w)
+        roof["prep"] = {name: {"ms": round(kern_ms[name], 5), "algorithmic_bytes": pb,
+                               "gbs": round(pb / (kern_ms[name] * 1e-3) / 1e9, 1),
+                               "frac_of_hbm": round(pb / (kern_ms[name] * 1e-3) / 1e9 / hbm, 4)}
+                        for name in ("fp8_rotate_quantize", "fp8_quantize") if name in kern_ms}
+    return roof
+
+
+def fp8_gemm_burst_tflops(dev, n=8192, reps=10):
+    """Measured dense E4M3 GEMM rate (library GEMM, torch._scaled_mm, n^3, best of
+    `reps`), the FP8 counterpart of the measured bf16 burst peak."""
+    import torch
+    try:
+        a = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device=dev).to(torch.float8_e4m3fn)
+        one = torch.ones((), device=dev, dtype=torch.float32)
+        best = float("inf")
+        for _ in range(reps + 2):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            best = min(best, e0.elapsed_time(e1))
+        del a, b
+        return round(2.0 * n ** 3 / (best * 1e-3) / 1e12, 1)
+    except Exception:
+        return None
+
+
 def run_ours(args):
     import torch
     rank, world, local = dist_env()
@@ -337,10 +507,11 @@ def run_ours(args):
     stream = torch.cuda.Stream(dev)
     step = Step(lib, w, x, dev)
     with ClockSampler(gpu_smi_id(dev, local)) as clk:
-        ms_rank = time_device(step, stream, args.steps, max(3, args.warmup), world, dev, clk)
+        ms_rank, kern_ms = time_device(step, stream, args.steps, max(3, args.warmup), world, dev, clk)
     st = lib.attn_get_device_status(stream.cuda_stream)
     if st != lib.ATTN_OK:
         raise lib.AttnError(st, "device status")
+    clocks = clk.summary()
     ms_total = max_over_ranks(ms_rank, world, dev)
     ms_step = ms_total / args.steps
     flops_rank = w.flops
@@ -352,37 +523,14 @@ def run_ours(args):
         e2e_ms = max_over_ranks(e2e_ms, world, dev)
         e2e = {"value": round(flops_rank * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
-    peak, hbm, peak_src = measured_peaks()
+    dt = "fp8" if w.fp8 else "bf16"
+    roof = roofline(w, kern_ms, clocks.get("sm_mhz"), args.workload)
     if w.fp8:
-        peak = peak * 2  # FP8 dense = 2x BF16 (nominal ratio)
-    # the dominant kernel is the attention kernel (one launch per BF16 step)
-    kernel_ms = ms_rank / args.steps
-    achieved = flops_rank / (kernel_ms * 1e-3) / 1e12
-    if w.N < 1024 and not w.fp8:
-        # small N (ViT shapes): arithmetic intensity below the ridge point, so the
-        # roofline is HBM: algorithmic bytes = Q, K, V read once + O written (bf16) + LSE (fp32)
-        bytes_launch = 2 * w.B * w.H * w.N * w.d * 4 + 4 * w.B * w.H * w.N
-        gbs = bytes_launch / (kernel_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(gbs / hbm, 4), "traffic": traffic_per_launch(args.workload),
-                "peak_source": f"{peak_src} copy bandwidth", "kernel": "attn_fwd_sm100",
-                "algorithmic_bytes": bytes_launch}
-    else:
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(args.workload),
-                "peak_source": f"{peak_src} bf16 burst" + (" x2 (fp8 nominal ratio)" if w.fp8 else ""),
-                "kernel": "attn_fwd_sm100" + ("+fp8_rotate_quantize" if w.fp8 else "")}
-    sus = sustained_bf16_peak()
-    if sus and roof["bound"] == "tensor":
-        # the timed loop runs long enough to meet the 1 kW power cap (see "clocks"); the
-        # sustained GEMM rate is the same-conditions denominator
-        sus = sus * 2 if w.fp8 else sus
-        roof["frac_of_sustained_peak"] = round(achieved / sus, 4)
-        roof["sustained_peak"] = sus
+        roof["measured_fp8_gemm_burst_tflops"] = fp8_gemm_burst_tflops(dev)
     cpu = None
     if rank == 0 and world == 1:
         cpu = cpu_baseline(w, budget_s=float(os.environ.get("ATTN_CPU_BASELINE_S", "15")))
-    clocks = clk.summary()
+    mhz = clocks.get("sm_mhz")
     line = {
         "metric": METRIC, "value": round(tflops, 3), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 5), "higher_is_better": True,
@@ -393,8 +541,13 @@ def run_ours(args):
                    "l2": "inputs larger than L2 (no flush)" if step.copies == 1 else
                    f"inputs smaller than L2: the timed loop rotates through {step.copies} copies "
                    f"(working set >= 2x L2, no flush)"},
-        "pct_of_peak": round(100 * tflops / world / peak, 2),
+        # the step's throughput against the datasheet dense tensor-core peak of the step's type
+        "pct_of_peak": round(100 * tflops / world / DATASHEET_TFLOPS[dt], 2),
+        "pct_of_peak_basis": f"B200 datasheet dense {dt.upper()} {DATASHEET_TFLOPS[dt]:.0f} TFLOP/s",
+        "pct_of_measured_peak": round(100 * tflops / world / (measured_peaks()[0] * (2 if w.fp8 else 1)), 2),
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": step.launches * args.steps,
+        "kernel_ms": {k: round(v, 5) for k, v in kern_ms.items()},
+        "cycles_per_step": None if mhz is None else round(ms_step * 1e-3 * mhz * 1e6),
         "clocks": clocks,
     }
     if rank == 0:

@@ -121,8 +121,21 @@ def _expect(t, name, shape, dtype, device):
         raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
 
 
-def forward(q, k, v, causal=False, scale=None, out=None, lse=None, with_lse=True, stream=None):
-    """O, LSE = attention(q, k, v) for bf16 CUDA tensors [B, H, N, d]."""
+def _check_device(check, stream_ptr, where):
+    """With check=True, wait for the launch and read the library's device status
+    word (one per device, shared by every stream and thread: a timeout of any
+    earlier launch is reported here too)."""
+    if check:
+        _check(attn_get_device_status(stream_ptr), where + " (device status)")
+
+
+def forward(q, k, v, causal=False, scale=None, out=None, lse=None, with_lse=True, stream=None, check=False):
+    """O, LSE = attention(q, k, v) for bf16 CUDA tensors [B, H, N, d].
+
+    The call is asynchronous. The outputs are valid once the launch has finished
+    AND attn_get_device_status() reports ATTN_OK (a pipeline wait that timed out
+    leaves them undefined); check=True does both before returning. `scale`
+    None selects 1/sqrt(d); a negative scale raises AttnError."""
     import torch
     B, H, N, d = _shape4(q)
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -135,8 +148,10 @@ def forward(q, k, v, causal=False, scale=None, out=None, lse=None, with_lse=True
     if lse is not None:
         _expect(lse, "lse", (B, H, N), torch.float32, q.device)
     sc = 0.0 if scale is None else float(scale)
+    sp = _stream_ptr(q, stream)
     _check(attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc,
-                    int(bool(causal)), ATTN_BF16, _stream_ptr(q, stream)), "attn_fwd")
+                    int(bool(causal)), ATTN_BF16, sp), "attn_fwd")
+    _check_device(check, sp, "attn_fwd")
     return out, lse
 
 
@@ -155,8 +170,11 @@ def quantize_fp8(x, rot=None, stream=None):
 
 
 def forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale=None, out=None, lse=None,
-                with_lse=True, stream=None):
-    """O (bf16), LSE from E4M3 codes and their per-tile scales."""
+                with_lse=True, stream=None, check=False):
+    """O (bf16), LSE from E4M3 codes and their per-tile scales (finite, >= 0).
+
+    Asynchronous like forward(): the outputs are valid once the launch has
+    finished and attn_get_device_status() reports ATTN_OK; check=True does both."""
     import torch
     B, H, N, d = _shape4(q8)
     T = (N + TILE - 1) // TILE
@@ -172,9 +190,11 @@ def forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale=None,
     if lse is not None:
         _expect(lse, "lse", (B, H, N), torch.float32, q8.device)
     sc = 0.0 if scale is None else float(scale)
+    sp = _stream_ptr(q8, stream)
     _check(attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_scale.data_ptr(), k_scale.data_ptr(),
-                        v_scale.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc, int(bool(causal)),
-                        _stream_ptr(q8, stream)), "attn_fwd_fp8")
+                        v_scale.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc, int(bool(causal)), sp),
+           "attn_fwd_fp8")
+    _check_device(check, sp, "attn_fwd_fp8")
     return out, lse
 
 

@@ -96,6 +96,15 @@ bool set_smem_once(const void* func, int bytes, int tag) {
 template <int D, bool FP8>
 constexpr int fwd_tag() { return FP8 ? 2 : (D == 128 ? 0 : 1); }
 
+// scale == 0 selects 1/sqrt(d); negative or non-finite scales are rejected
+// (the kernels take the row maximum of scale * Q K^T through the maximum of
+// Q K^T, which only holds for a positive scale).
+attn_status resolve_scale(float& scale, int d) {
+  if (!std::isfinite(scale) || scale < 0.f) return ATTN_ERR_INVALID_ARG;
+  if (scale == 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
+  return ATTN_OK;
+}
+
 attn_status check_shape(int B, int H, int N) {
   if (B < 1 || H < 1 || N < 1) return ATTN_ERR_INVALID_ARG;
   const long long rows = static_cast<long long>(B) * H * N;
@@ -121,10 +130,15 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.BH = BH;
   p.num_units = BH * npair;
   // Non-causal: heads per group such that the group's K and V (2 N d bytes per
-  // element per head) take about 48 MB of the 126 MB L2. Causal: all heads.
+  // element per head) take about 48 MB of the 126 MB L2. Causal: all heads
+  // unless ATTN_CAUSAL_GROUP_MB gives a budget for causal groups too.
+#ifndef ATTN_CAUSAL_GROUP_MB
+#define ATTN_CAUSAL_GROUP_MB 0
+#endif
   {
     const long long kv_bytes = 2ll * N * C::D * (C::FP8 ? 1 : 2);
-    long long hg = causal ? BH : (48ll << 20) / (kv_bytes > 0 ? kv_bytes : 1);
+    const long long budget = causal ? (static_cast<long long>(ATTN_CAUSAL_GROUP_MB) << 20) : (48ll << 20);
+    long long hg = budget == 0 ? BH : budget / (kv_bytes > 0 ? kv_bytes : 1);
     if (hg < 1) hg = 1;
     if (hg > BH) hg = BH;
     p.heads_per_group = static_cast<int>(hg);
@@ -170,16 +184,15 @@ const char* attn_status_string(int status) {
 }
 
 attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                     float scale, int causal, int dtype, void* stream) {
+                     float scale, int causal, attn_dtype dtype, void* stream) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = resolve_scale(scale, d); s != ATTN_OK) return s;
   if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
   if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
     return ATTN_ERR_MISALIGNED;
-  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
   if (d == 128)
@@ -192,13 +205,12 @@ attn_status attn_fwd_inject_timeout(const void* q, const void* k, const void* v,
                                     unsigned long long wait_limit_cycles, void* stream) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = resolve_scale(scale, d); s != ATTN_OK) return s;
   if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
   if (d != 128) return ATTN_ERR_UNSUPPORTED;
   if (fault_unit < 0 || wait_limit_cycles < 1024) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
     return ATTN_ERR_MISALIGNED;
-  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
   return launch_fwd<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, B * H, N, scale, causal,
                                 static_cast<cudaStream_t>(stream), fault_unit, wait_limit_cycles);
 }
@@ -210,12 +222,11 @@ attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const f
       k_scale == nullptr || v_scale == nullptr)
     return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = resolve_scale(scale, d); s != ATTN_OK) return s;
   if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
   if (d != 128) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
     return ATTN_ERR_MISALIGNED;
-  if (scale <= 0.f) scale = 1.0f / std::sqrt(static_cast<float>(d));
   return launch_fwd<128, true>(q8, k8, v8, o, lse, q_scale, k_scale, v_scale, B * H, N, scale, causal,
                                static_cast<cudaStream_t>(stream));
 }

@@ -648,8 +648,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tmem_ld_wait<128>(sr);
         float c = p.scale_log2, v_log2_ratio = 0.f;
         if constexpr (C::FP8) {
-          c *= q_sc * p.k_scale[bh * T + j];
-          v_log2_ratio = __log2f(p.v_scale[bh * T + j] / v_max);
+          // A tile scale of 0 (a tile that dequantises to zeros) must not turn
+          // the row into NaN: the score factor is kept positive (the scores
+          // of such a tile are then ~0, as they should be) and the V ratio at
+          // or above 2^-64 (its P rounds to zero in E4M3; the fp32 row sum
+          // keeps its exact share of the normaliser).
+          c = fmaxf(c * (q_sc * p.k_scale[bh * T + j]), 1e-30f);
+          v_log2_ratio = __log2f(fmaxf(p.v_scale[bh * T + j] / v_max, 5.421010862427522e-20f));
         }
         // masking: causal diagonal block and the ragged last key block
         const bool masked = (j == nkv_t - 1) && (p.causal || (p.N % kBlockN) != 0);

@@ -19,12 +19,20 @@
  *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed as
  *     void*, NULL = the legacy default stream). The host never synchronises.
  *   - Causal masking is square and top-left aligned: query i sees keys j <= i.
- *   - scale <= 0 selects the default 1/sqrt(d).
+ *   - scale == 0 selects the default 1/sqrt(d) (eq. Scores); a negative or
+ *     non-finite scale is an argument error.
  *   - Argument errors are detected on the host before anything is launched and
  *     returned immediately (INVALID_ARG, UNSUPPORTED, MISALIGNED). A failed
  *     launch returns ATTN_ERR_CUDA. A device-side pipeline wait that exceeds its
  *     time limit makes the kernel stop early and record ATTN_ERR_TIMEOUT in a
  *     device status word, read by attn_get_device_status().
+ *   - A returned ATTN_OK means the launch was queued. The outputs are valid
+ *     only once attn_get_device_status() has returned ATTN_OK after the launch
+ *     completed: a launch that timed out leaves them undefined.
+ *   - The status word is ONE word per device for the whole library, shared by
+ *     every stream, thread and entry point: a timeout recorded by a launch on
+ *     stream A is reported (and cleared) by whichever attn_get_device_status()
+ *     call reads it first, whatever stream that call names.
  *   - N >= 1, B >= 1, H >= 1, and B*H*N < 2^31.
  */
 #ifndef ATTN_B200_H
@@ -49,6 +57,7 @@ typedef enum {
   ATTN_ERR_TIMEOUT = 5       /* a device pipeline wait ran out (see below)       */
 } attn_status;
 
+/* Element type of attn_fwd's q, k, v and o (passed as an int-sized enum). */
 typedef enum {
   ATTN_BF16 = 0              /* bf16 inputs and output, fp32 accumulation        */
 } attn_dtype;
@@ -67,7 +76,7 @@ typedef enum {
  * FlashAttention-3 asynchronous copies and warp specialisation).
  */
 ATTN_API attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                     int B, int H, int N, int d, float scale, int causal, int dtype,
+                     int B, int H, int N, int d, float scale, int causal, attn_dtype dtype,
                      void* stream);
 
 /*
@@ -88,15 +97,24 @@ ATTN_API attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8,
                               int B, int H, int N, int d, void* stream);
 
 /*
- * attn_fwd_fp8 - attention forward on block-quantised E4M3 inputs.
+ * attn_fwd_fp8 - attention forward on block-quantised E4M3 inputs
+ * ("FlashAttention scaling, multi-GPU training and weight quantization",
+ * section 1, FlashAttention-3 FP8 bullet: FP8 tensor-core inputs with one scale
+ * per small tile, Q and K made incoherent by a random orthogonal matrix; what
+ * is computed is the attention of "Self-Attention, CUDA kernels and
+ * FlashAttention", section 1, eq. Attention, on the dequantised values).
  *   q8, k8, v8 : [B, H, N, d] E4M3 codes (q8, k8 rotated by the same orthogonal
  *                matrix, which leaves Q K^T unchanged).
  *   q_scale, k_scale, v_scale : [B, H, ceil(N/128)] fp32 tile scales; the
  *                value of a code is decode(code) * scale of its 128-token tile.
+ *                Every scale must be finite and >= 0 (attn_quantize_fp8 writes
+ *                only positive ones); a tile whose scale is 0 dequantises to
+ *                zeros. The library cannot check device arrays on the host:
+ *                a negative, infinite or NaN scale gives an undefined result.
  *   o   : [B, H, N, d] bf16 output.  lse: [B, H, N] fp32 or NULL.
  *   d   : 128 (else ATTN_ERR_UNSUPPORTED).
- * Computes the attention of the dequantised values; P is re-quantised to E4M3
- * on chip for the P V product (the error this adds is within the FP8 tolerance).
+ * P is re-quantised on chip for the P V product (two E4M3 terms per value);
+ * the error this adds is within the FP8 tolerance of the tests.
  */
 ATTN_API attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
                          const float* q_scale, const float* k_scale, const float* v_scale,

@@ -71,6 +71,8 @@ def test_fwd_argument_validation(lib):
     assert call(B=-1) == lib.ATTN_ERR_INVALID_ARG
     assert call(causal=2) == lib.ATTN_ERR_INVALID_ARG
     assert call(scale=float("nan")) == lib.ATTN_ERR_INVALID_ARG
+    assert call(scale=float("inf")) == lib.ATTN_ERR_INVALID_ARG
+    assert call(scale=-0.125) == lib.ATTN_ERR_INVALID_ARG    # only 0 selects the default
     assert call(B=1 << 16, H=1 << 10, N=1 << 10) == lib.ATTN_ERR_INVALID_ARG  # rows overflow int32
     assert call(d=96) == lib.ATTN_ERR_UNSUPPORTED
     assert call(d=256) == lib.ATTN_ERR_UNSUPPORTED
@@ -86,6 +88,9 @@ def test_fp8_argument_validation(lib):
     args = list(base)
     args[11] = 64
     assert f(*args) == lib.ATTN_ERR_UNSUPPORTED
+    args = list(base)
+    args[12] = -1.0
+    assert f(*args) == lib.ATTN_ERR_INVALID_ARG
     args = list(base)
     args[2] = FAKE + 1
     assert f(*args) == lib.ATTN_ERR_MISALIGNED

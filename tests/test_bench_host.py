@@ -7,7 +7,8 @@ ROW = "{sm}, 1965, 900, Not Active, Not Active, Not Active, {cap}"
 
 def _sampler(samples, window):
     c = bench.ClockSampler("0")
-    c.lines = [(t, ROW.format(sm=sm, cap="Active" if cap else "Not Active")) for t, sm, cap in samples]
+    c.samples = [bench.ClockSampler.parse_smi_line(t, ROW.format(sm=sm, cap="Active" if cap else "Not Active"))
+                 for t, sm, cap in samples]
     c.window = window
     return c
 
@@ -29,6 +30,32 @@ def test_summary_falls_back_to_all_samples():
 
 def test_summary_without_samples():
     assert _sampler([], None).summary()["samples"] == 0
+
+
+def test_smi_line_parsing():
+    assert bench.ClockSampler.parse_smi_line(0.0, "garbage") is None
+    t, sm, mx, r = bench.ClockSampler.parse_smi_line(1.0, "1500, 1965, 990.1, Active, Not Active, Not Active, Active")
+    assert (sm, mx, r) == (1500.0, 1965.0, {"hw_slowdown", "sw_power_cap"})
+
+
+def test_roofline_denominators():
+    """The attention kernel's roofline uses its own mean launch time; the hardware
+    peak at the sampled clock is 148 SMs x 8192 bf16 FLOP per clock."""
+    import workloads
+    w = workloads.WORKLOADS["llm_train_causal"]
+    ms = w.flops / 1000e12 * 1e3          # a launch time giving exactly 1000 TFLOP/s
+    r = bench.roofline(w, {"attn_fwd_sm100": ms}, 1965.0, w.name)
+    assert r["bound"] == "tensor" and abs(r["achieved"] - 1000.0) < 1e-6
+    assert abs(r["hw_peak_at_sampled_clock"] - 148 * 8192 * 1965e6 / 1e12) < 0.1
+    assert abs(r["frac_of_datasheet_peak"] - 1000 / 2250) < 1e-4
+    wv = workloads.WORKLOADS["vit_b16_batch"]
+    rv = bench.roofline(wv, {"attn_fwd_sm100": 0.05}, None, wv.name)
+    assert rv["bound"] == "hbm" and rv["unit"] == "GB/s"
+    wf = workloads.WORKLOADS["fp8_rotated"]
+    rf = bench.roofline(wf, {"attn_fwd_sm100": 1.0, "fp8_rotate_quantize": 0.1, "fp8_quantize": 0.05}, 1800.0,
+                        wf.name)
+    assert set(rf["prep"]) == {"fp8_rotate_quantize", "fp8_quantize"}
+    assert rf["prep"]["fp8_quantize"]["algorithmic_bytes"] == 2 * 32 * 8192 * 128 * 3 + 4 * 2 * 32 * 64
 
 
 def test_reference_arm_prints_one_contract_line():

@@ -125,12 +125,27 @@ def test_zero_query_and_zero_scale(causal):
 
 @pytest.mark.parametrize("causal", [False, True])
 def test_probability_rows_sum_to_one(causal):
-    q, k = RNG.standard_normal((2, 3, 50, 16)), RNG.standard_normal((2, 3, 50, 16))
-    p = attention_probs_fp64(q, k, 0.25, causal)
+    """Rows of the materialised P sum to 1 ("Self-Attention, CUDA kernels and
+    FlashAttention", §1, softmax paragraph), and that P is the one behind the
+    oracle's outputs: P V equals attention_fp64's O and ln P_ij + LSE_i equals
+    the score S_ij written out with explicit loops (a dropped scale or a
+    transposed product in either function fails here)."""
+    B, H, N, d = 2, 3, 50, 16
+    q, k, v = (RNG.standard_normal((B, H, N, d)) for _ in range(3))
+    scale = 0.25
+    p = attention_probs_fp64(q, k, scale, causal)
     np.testing.assert_allclose(p.sum(-1), 1.0, atol=1e-13)
     assert (p >= 0).all()
     if causal:
         assert np.all(np.triu(p[0, 0], 1) == 0)
+    o, lse = attention_fp64(q, k, v, scale, causal)
+    np.testing.assert_allclose(np.einsum("bhij,bhjc->bhic", p, v), o, rtol=0, atol=1e-12)
+    for b, h, i, j in ((0, 0, 3, 1), (1, 2, 49, 0), (1, 1, 20, 20), (0, 2, 7, 30)):
+        if causal and j > i:
+            assert p[b, h, i, j] == 0.0
+            continue
+        s_ij = scale * sum(q[b, h, i, t] * k[b, h, j, t] for t in range(d))
+        assert abs(math.log(p[b, h, i, j]) + lse[b, h, i] - s_ij) <= 1e-12
 
 
 @pytest.mark.parametrize("causal", [False, True])

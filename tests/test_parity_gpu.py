@@ -123,7 +123,7 @@ def test_bf16_lse_optional(cuda_lib):
 
 
 # ---------------------------------------------------------------- full-size workloads
-BF16_WORKLOADS = ["vit_b16_single", "vit_b16_batch", "llm_train_causal", "long_seq_causal"]
+BF16_WORKLOADS = ["vit_b16_single", "vit_b16_batch", "llm_train_causal", "long_seq_causal", "noncausal_8k_bf16"]
 
 
 @pytest.mark.parametrize("name", BF16_WORKLOADS)
@@ -213,7 +213,22 @@ def fp8_reference(q, k, v, rot, scale, causal, rows=None, heads=None):
     return o, l, (qc[0], qs[0], kc[0], ks[0], vc[0], vs[0])
 
 
-@pytest.mark.parametrize("shape", [(1, 1, 128, 128), (1, 2, 300, 128), (2, 1, 1000, 128), (1, 1, 17, 128)],
+def run_fp8(lib, q8, k8, v8, qs, ks, vs, causal):
+    """attn_fwd_fp8 into NaN-prefilled, canary-fenced O and LSE; the canaries and
+    the device status word are checked after the launch."""
+    dev = torch.device("cuda:0")
+    B, H, N, d = q8.shape
+    o = Guarded((B, H, N, d), torch.bfloat16, dev)
+    lse = Guarded((B, H, N), torch.float32, dev)
+    lib.forward_fp8(q8, k8, v8, qs, ks, vs, causal=causal, out=o.t, lse=lse.t)
+    torch.cuda.synchronize()
+    assert o.canaries_intact() and lse.canaries_intact(), "write outside the output"
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+    return o.t.float().cpu().numpy(), lse.t.cpu().numpy()
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 128, 128), (1, 2, 300, 128), (2, 1, 1000, 128), (1, 1, 17, 128),
+                                   (1, 1, 1, 128), (2, 3, 257, 128)],
                          ids=lambda s: "x".join(map(str, s)))
 @pytest.mark.parametrize("causal", [False, True])
 def test_fp8_small_parity(cuda_lib, shape, causal):
@@ -221,14 +236,52 @@ def test_fp8_small_parity(cuda_lib, shape, causal):
     q, k, v = workloads.make_qkv(B, H, N, d, seed=N + 5, outliers=("q", "k", "v"))
     rot = workloads.make_rotation(d, 17)[1]
     q8, k8, v8, qs, ks, vs = fp8_inputs(cuda_lib, q, k, v, rot)
-    o, lse = cuda_lib.forward_fp8(q8, k8, v8, qs, ks, vs, causal=causal)
-    torch.cuda.synchronize()
+    o, lse = run_fp8(cuda_lib, q8, k8, v8, qs, ks, vs, causal)
     o_ref, l_ref, _ = fp8_reference(q, k, v, rot, 1 / math.sqrt(d), causal)
-    o = o.float().cpu().numpy().reshape(B * H, N, d)
-    lse = lse.cpu().numpy().reshape(B * H, N)
-    assert np.isfinite(o).all()
+    o = o.reshape(B * H, N, d)
+    lse = lse.reshape(B * H, N)
+    assert np.isfinite(o).all(), "NaN/inf in O (unwritten element?)"
+    assert np.isfinite(lse).all(), "NaN/inf in LSE"
     assert np.abs(o - o_ref).max() <= TOL_FP8
     assert np.abs(lse - l_ref).max() <= TOL_LSE
+
+
+def test_fp8_zero_scale_tiles(cuda_lib):
+    """Tiles whose scale is 0 dequantise to zeros: a zero V tile contributes
+    nothing and a zero K tile gives scores of exactly 0, with no NaN anywhere."""
+    B, H, N, d = 1, 2, 384, 128
+    q, k, v = workloads.make_qkv(B, H, N, d, seed=404)
+    rot = workloads.make_rotation(d, 17)[1]
+    q8, k8, v8, qs, ks, vs = fp8_inputs(cuda_lib, q, k, v, rot)
+    vs[0, 0, 1] = 0.0            # head 0: V tile 1 is zero
+    ks[0, 1, 2] = 0.0            # head 1: K tile 2 is zero
+    vs[0, 1, 0] = 0.0            # head 1: V tile 0 is zero too
+    for causal in (False, True):
+        o, lse = run_fp8(cuda_lib, q8, k8, v8, qs, ks, vs, causal)
+        assert np.isfinite(o).all() and np.isfinite(lse).all()
+        codes = [x.cpu().numpy() for x in (q8, k8, v8)]
+        scs = [x.cpu().numpy() for x in (qs, ks, vs)]
+        qd, kd, vd = (dequantize(c, sc) for c, sc in zip(codes, scs))
+        o_ref, l_ref = attention_fp64(qd, kd, vd, 1 / math.sqrt(d), causal)
+        assert np.abs(o - o_ref).max() <= TOL_FP8
+        assert np.abs(lse - l_ref).max() <= TOL_LSE
+
+
+def test_fp8_deterministic(cuda_lib):
+    q, k, v = workloads.make_qkv(2, 3, 700, 128, seed=19, outliers=("q", "k", "v"))
+    rot = workloads.make_rotation(128, 17)[1]
+    q8, k8, v8, qs, ks, vs = fp8_inputs(cuda_lib, q, k, v, rot)
+    for causal in (False, True):
+        outs = [cuda_lib.forward_fp8(q8, k8, v8, qs, ks, vs, causal=causal) for _ in range(5)]
+        torch.cuda.synchronize()
+        for o, l in outs[1:]:
+            assert torch.equal(o.view(torch.int16), outs[0][0].view(torch.int16))
+            assert torch.equal(l.view(torch.int32), outs[0][1].view(torch.int32))
+    # the preparation kernel is deterministic as well
+    again = fp8_inputs(cuda_lib, q, k, v, rot)
+    torch.cuda.synchronize()
+    for a, b in zip((q8, k8, v8, qs, ks, vs), again):
+        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8))
 
 
 def test_fp8_workload_parity(cuda_lib):
@@ -238,6 +291,7 @@ def test_fp8_workload_parity(cuda_lib):
     o, lse = cuda_lib.forward_fp8(q8, k8, v8, qs, ks, vs, causal=w.causal)
     torch.cuda.synchronize()
     assert cuda_lib.attn_get_device_status(None) == cuda_lib.ATTN_OK
+    assert bool(torch.isfinite(o.float()).all()) and bool(torch.isfinite(lse).all())
     heads = list(range(0, w.B * w.H, 8))
     rows = workloads.sample_rows(w.N, 96, w.seed)
     o_ref, l_ref, ref_codes = fp8_reference(x["q"], x["k"], x["v"], x["rot"], w.scale, w.causal, rows=rows,
