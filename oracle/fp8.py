@@ -12,16 +12,25 @@ without rotation.
 Readings (the page gives no numbers, so these are this library's definitions,
 shared with the CUDA kernels only through this specification, not through code):
   * tile = 128 consecutive tokens x all d channels of one (batch, head);
-  * rotated value y = x R accumulated in fp32 in increasing k order; every
-    product of two bf16 values is exact in fp32, so the result is unique;
+  * rotated value y = x R, the plain matrix product: computed here in fp64
+    (every product of two bf16 values is exact there, the sums carry errors of
+    order 2^-45 relative) and rounded once to fp32. The page fixes "multiply by
+    a random orthogonal matrix", not an accumulation order or precision, so a
+    tensor-core product with fp32 accumulation is an equally valid computation
+    of y: its result differs from this one by fp32 accumulation error only;
   * scale = amax(|y| over the tile) / 448 in fp32 (IEEE division); a tile of all
     zeros gets scale 1;
-  * code = E4M3(y / scale), fp32 IEEE division, then round-to-nearest-even to
-    OCP E4M3 with saturation to +-448 (the format's largest finite value);
+  * code = E4M3(y * r), r = 1 / scale in fp32 (one IEEE division per tile), the
+    product rounded to fp32, then round-to-nearest-even to OCP E4M3 with
+    saturation to +-448 (the format's largest finite value);
   * dequantised value = decode(code) * scale, which is what the attention
     oracle consumes.
-Because a float decides an integer code here, the oracle takes that decision
-in the same precision as the kernel (fp32), so codes are compared bit-exactly.
+Where a float decides an integer code, the decision is taken in fp32, the
+kernel's precision. Without rotation (V) y = x exactly, so codes and scales are
+unique and compare bit for bit; with rotation the kernel's y may differ from
+the exact product by its accumulation error, which can move a code by one step
+where y * r lies within that error of a rounding boundary (the GPU tests bound
+where and how often).
 
 E4M3 (OCP 8-bit floating point, E4M3 variant): 1 sign bit, 4 exponent bits with
 bias 7, 3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; the code
@@ -79,17 +88,13 @@ def e4m3_encode(x):
     return code.astype(np.uint8)
 
 
-def rotate_fp32(x_bf16_as_f32, rot_bf16_as_f32):
-    """y = x R in fp32, each output accumulated in increasing k order.
+def rotate(x_bf16_as_f32, rot_bf16_as_f32):
+    """y = x R: the exact product (fp64: bf16 products are exact, the sums are
+    within ~2^-45 relative) rounded once to fp32.
     x: [..., d] float32 holding bf16 values; rot: [d, d] float32 holding bf16."""
-    x = np.asarray(x_bf16_as_f32, dtype=np.float32)
-    r = np.asarray(rot_bf16_as_f32, dtype=np.float32)
-    d = x.shape[-1]
-    y = np.zeros(x.shape[:-1] + (r.shape[1],), dtype=np.float32)
-    for kk in range(d):
-        # product of two bf16 values is exact in fp32; one rounding per add
-        y += x[..., kk:kk + 1] * r[kk:kk + 1, :]
-    return y
+    x = np.asarray(x_bf16_as_f32, dtype=np.float64)
+    r = np.asarray(rot_bf16_as_f32, dtype=np.float64)
+    return (x @ r).astype(np.float32)
 
 
 def quantize_tiles(y_f32):
@@ -105,7 +110,8 @@ def quantize_tiles(y_f32):
         amax = np.abs(blk).reshape(BH, -1).max(axis=1).astype(np.float32)
         sc = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
         scales[:, t] = sc
-        q = (blk / sc[:, None, None]).astype(np.float32)   # fp32 IEEE division
+        inv = (np.float32(1.0) / sc).astype(np.float32)           # fp32 IEEE division, once per tile
+        q = (blk * inv[:, None, None]).astype(np.float32)         # fp32 product, rounded once
         codes[:, t * TILE:(t + 1) * TILE, :] = e4m3_encode(q)
     return codes, scales
 
@@ -119,7 +125,7 @@ def prepare_fp8(x_bf16, rot_bf16=None):
     x = _to_f32(x_bf16)
     B, H, N, d = x.shape
     x = x.reshape(B * H, N, d)
-    y = x if rot_bf16 is None else rotate_fp32(x, _to_f32(rot_bf16))
+    y = x if rot_bf16 is None else rotate(x, _to_f32(rot_bf16))
     codes, scales = quantize_tiles(y)
     return codes.reshape(B, H, N, d), scales.reshape(B, H, -1)
 

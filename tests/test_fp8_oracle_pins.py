@@ -5,10 +5,12 @@
     even code;
   * the encoder agrees with torch's float8_e4m3fn conversion (a library routine)
     on random values after clamping to +-448;
-  * the fp32 rotation equals an fp64 product rounded once per step, and is exact
-    for a permutation matrix;
+  * the rotation equals the exact rational product rounded once to fp32, and is
+    exact for a permutation matrix;
   * block scales: amax of the tile maps to 448, zeros give scale 1, dequantised
-    values are within half a code step of the input.
+    values are within half a code step of the input;
+  * the quantiser multiplies by the fp32 reciprocal of the tile scale (a value
+    worked by hand where dividing instead would give the neighbouring code).
 """
 import json
 import os
@@ -17,7 +19,9 @@ import numpy as np
 import pytest
 import torch
 
-from oracle import e4m3_decode, e4m3_encode, prepare_fp8, dequantize, rotate_fp32
+from fractions import Fraction
+
+from oracle import e4m3_decode, e4m3_encode, prepare_fp8, dequantize, rotate
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -60,24 +64,55 @@ def test_encoder_matches_torch_float8():
     np.testing.assert_array_equal(got, ref)
 
 
-def test_rotation_fp32_is_sequential_and_exact_products():
+def _fp32_round(v: Fraction) -> float:
+    """Exact rational -> nearest fp32 (ties to even), for normal magnitudes."""
+    if v == 0:
+        return 0.0
+    a = abs(v)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    quantum = Fraction(2) ** (e - 23)
+    n = round(a / quantum)                 # Fraction.__round__: half to even
+    r = float(n * quantum)
+    return r if v > 0 else -r
+
+
+def test_rotation_is_the_exact_product_rounded_once():
     rng = np.random.default_rng(3)
     d = 16
     x = torch.from_numpy(rng.standard_normal((5, d)).astype(np.float32)).to(torch.bfloat16)
     r = torch.from_numpy(rng.standard_normal((d, d)).astype(np.float32) / 4).to(torch.bfloat16)
-    y = rotate_fp32(x.float().numpy(), r.float().numpy())
-    # independent restatement: fp64 products (exact), fp32 rounding after each add
+    y = rotate(x.float().numpy(), r.float().numpy())
+    assert y.dtype == np.float32
+    # independent restatement: exact rational sum of the (bf16) products, one rounding
     xf, rf = x.double().numpy(), r.double().numpy()
     for i in range(5):
         for c in range(d):
-            acc = np.float32(0.0)
-            for kk in range(d):
-                acc = np.float32(np.float64(acc) + xf[i, kk] * rf[kk, c])
-            assert y[i, c] == acc
+            exact = sum(Fraction(float(xf[i, kk])) * Fraction(float(rf[kk, c])) for kk in range(d))
+            assert float(y[i, c]) == _fp32_round(exact), (i, c)
     # a permutation matrix moves values exactly
     perm = np.eye(d, dtype=np.float32)[rng.permutation(d)]
-    yp = rotate_fp32(x.float().numpy(), perm)
+    yp = rotate(x.float().numpy(), perm)
     np.testing.assert_array_equal(yp, x.float().numpy() @ perm)
+
+
+def test_quantiser_multiplies_by_the_fp32_reciprocal():
+    """Worked by hand. A tile whose largest magnitude is 3136 = 7 * 448 has the
+    scale 3136 / 448 = 7 exactly; r = fp32(1/7) = 0.142857149... is 4.5e-8 too
+    large (relative). The value 10.9375 = 7 * 1.5625 sits, after exact division,
+    on the midpoint 1.5625 between the E4M3 values 1.5 (code 0x3C, even mantissa)
+    and 1.625 (0x3D), which ties to 0x3C; multiplied by r it becomes
+    fp32(1.5625 * (1 + 4.5e-8)) = 1.5625 + 2^-23, above the midpoint: 0x3D."""
+    x = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16)
+    x[0, 0, 0, 0] = 3136.0
+    x[0, 0, 5, 7] = 10.9375
+    x[0, 0, 9, 3] = -10.9375
+    codes, scales = prepare_fp8(x, None)
+    assert scales[0, 0, 0] == 7.0
+    assert codes[0, 0, 0, 0] == 0x7E            # 448
+    assert codes[0, 0, 5, 7] == 0x3D
+    assert codes[0, 0, 9, 3] == 0xBD
 
 
 def test_block_quantisation_properties():
@@ -118,3 +153,44 @@ def test_rotation_spreads_outliers():
     _, s_plain = prepare_fp8(xb, None)
     _, s_rot = prepare_fp8(xb, rot)
     assert s_rot[0, 0, 0] < 0.5 * s_plain[0, 0, 0]
+
+
+def _quantize_like_gpu(y32):
+    """Block quantisation of an fp32 y [BH, N, d] the way the reading defines it
+    (fp32 amax / 448, fp32 reciprocal, fp32 product, E4M3)."""
+    BH, N, d = y32.shape
+    T = (N + 127) // 128
+    codes = np.empty(y32.shape, np.uint8)
+    scales = np.empty((BH, T), np.float32)
+    for t in range(T):
+        blk = y32[:, t * 128:(t + 1) * 128]
+        amax = np.abs(blk).reshape(BH, -1).max(1)
+        s = np.where(amax > 0, amax / np.float32(448.0), np.float32(1.0)).astype(np.float32)
+        inv = (np.float32(1.0) / s).astype(np.float32)
+        scales[:, t] = s
+        codes[:, t * 128:(t + 1) * 128] = e4m3_encode((blk * inv[:, None, None]).astype(np.float32))
+    return codes, scales
+
+
+def test_rotated_code_bounds_admit_fp32_accumulation_and_reject_mistakes():
+    """The GPU check for rotated tensors (tests/fp8_bounds.py) accepts the codes of
+    any fp32 accumulation order of x R (here: increasing k, decreasing k) and the
+    oracle's own, and rejects a transposed rotation and a dropped rotation."""
+    from fp8_bounds import check_rotated
+    from workloads import make_qkv, make_rotation
+    q, _, _ = make_qkv(1, 2, 300, 128, seed=8, outliers=("q",))
+    x = q.reshape(2, 300, 128)
+    _, rot = make_rotation(128, 3)
+    xf, rf = x.float().numpy(), rot.float().numpy()
+    codes_o, scales_o = prepare_fp8(x.unsqueeze(0), rot)
+    assert check_rotated(x, rot, codes_o[0], scales_o[0]) == 0
+    for order in (range(128), range(127, -1, -1)):
+        y = np.zeros((2, 300, 128), np.float32)
+        for kk in order:
+            y = (y + xf[..., kk:kk + 1] * rf[kk:kk + 1, :]).astype(np.float32)
+        c, s = _quantize_like_gpu(y)
+        check_rotated(x, rot, c, s)
+    for wrong in (xf @ rf.T, xf):
+        c, s = _quantize_like_gpu(wrong.astype(np.float32))
+        with pytest.raises(AssertionError):
+            check_rotated(x, rot, c, s)

@@ -13,7 +13,7 @@ Workload shapes follow the pages:
     multiplied by a random orthogonal matrix before block quantisation
     ("FlashAttention scaling, multi-GPU training and weight quantization", §1,
     FlashAttention-3 FP8 bullet: block quantisation and incoherent processing).
-    The same shape and outliers also run in BF16 without quantisation.
+    The same shape also runs in BF16 without quantisation (outliers in Q and K).
 
 Recipe (all on the CPU, torch.Generator seeded per workload):
   1. Q, K, V drawn in that order as fp32 iid N(0, 1), shape [B, H, N, d].
@@ -67,10 +67,12 @@ WORKLOADS = {
                                 outliers=("q", "k"), seed=1003),
     "fp8_rotated": Workload("fp8_rotated", 2, 32, 8192, 128, False, fp8=True,
                             outliers=("q", "k", "v"), seed=1004),
-    # the FP8 workload's shape and outliers in BF16 (no quantisation): the
-    # non-causal N >= 4096, d = 128 shape of the tensor-core target
+    # the FP8 workload's shape in BF16 (no quantisation): the non-causal
+    # N >= 4096, d = 128 shape of the tensor-core target, with the BF16
+    # long-sequence recipe (outliers in Q and K only: with magnitude-20 V
+    # entries |O| reaches 20, where one bf16 step of the output is 0.125)
     "noncausal_8k_bf16": Workload("noncausal_8k_bf16", 2, 32, 8192, 128, False,
-                                  outliers=("q", "k", "v"), seed=1005),
+                                  outliers=("q", "k"), seed=1005),
 }
 
 OUTLIER_FRACTION = 0.001
