@@ -237,18 +237,34 @@ attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* s
   if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
   if (d != attn::kPrepTile) return ATTN_ERR_UNSUPPORTED;
   if (!aligned16(x) || !aligned16(x8) || (rot != nullptr && !aligned16(rot))) return ATTN_ERR_MISALIGNED;
+  const int BH = B * H;
   const int T = (N + attn::kPrepTile - 1) / attn::kPrepTile;
-  if (!set_smem_once(reinterpret_cast<const void*>(attn::fp8_rotate_quantize), attn::kPrepSmemBytes, 3))
+  // X tiles {128 rows of bf16 in two 64-column chunks}, R as one such tile, the
+  // codes as {128 rows x 128 bytes}; all with the 128-byte swizzle
+  CUtensorMap tx, tr, to;
+  if (!encode_qkv_map(&tx, x, false, d, N, BH, attn::kPrepTile) ||
+      !encode_qkv_map(&to, x8, true, d, N, BH, attn::kPrepTile) ||
+      !encode_qkv_map(&tr, rot != nullptr ? rot : x, false, d, rot != nullptr ? d : N, rot != nullptr ? 1 : BH,
+                      attn::kPrepTile))
     return ATTN_ERR_CUDA;
-  const int num_tiles = B * H * T;
+  const bool rotate = rot != nullptr;
+  const void* kern = rotate ? reinterpret_cast<const void*>(attn::fp8_prep_sm100<true>)
+                            : reinterpret_cast<const void*>(attn::fp8_prep_sm100<false>);
+  const int tag = rotate ? 3 : 4;
+  if (!set_smem_once(kern, attn::PrepCfg::SMEM_BYTES, tag)) return ATTN_ERR_CUDA;
+  const int num_tiles = BH * T;
   const int sms = sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
-  attn::fp8_rotate_quantize<<<num_tiles < sms ? num_tiles : sms, attn::kPrepThreads, attn::kPrepSmemBytes,
-                              static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(rot), static_cast<uint8_t*>(x8),
-      scales, N, num_tiles);
+  const int grid = num_tiles < sms ? num_tiles : sms;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (rotate)
+    attn::fp8_prep_sm100<true><<<grid, attn::PrepCfg::THREADS, attn::PrepCfg::SMEM_BYTES, st>>>(
+        tx, tr, to, scales, T, num_tiles, kWaitLimitCycles);
+  else
+    attn::fp8_prep_sm100<false><<<grid, attn::PrepCfg::THREADS, attn::PrepCfg::SMEM_BYTES, st>>>(
+        tx, tr, to, scales, T, num_tiles, kWaitLimitCycles);
   if (cudaGetLastError() != cudaSuccess) {
-    forget_smem(3);
+    forget_smem(tag);
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;

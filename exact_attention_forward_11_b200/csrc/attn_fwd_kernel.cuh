@@ -45,17 +45,12 @@
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
+#include "status.cuh"
 
 namespace attn {
 
 constexpr int kBlockM = 128;  // query rows per Q tile
 constexpr int kBlockN = 128;  // keys per K/V block
-constexpr uint32_t kStatusTimeout = 1u;
-
-// Device status word (global memory of this module). A kernel whose bounded
-// wait ran out ORs kStatusTimeout into it; attn_get_device_status reads and
-// clears it.
-__device__ uint32_t g_status;
 
 template <int D_, bool FP8_>
 struct FwdCfg {
@@ -149,8 +144,6 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint6
   }
   return true;
 }
-
-__device__ __forceinline__ void record_timeout() { atomicOr(&g_status, kStatusTimeout); }
 
 // 2^x for a pair of fp32 arguments on the FMA/ALU pipes. Cody-Waite style
 // reduction x = n + f with n = round(x) (adding 1.5 * 2^23 leaves n in the low
