@@ -1,9 +1,8 @@
 """CPU oracle (test infrastructure only).
 
 Plain, slow, fp64 restatement of what the attention forward and its backward
-pass compute, plus the
-FP8 preparation (exact rotation, block quantisation decided in the kernel's fp32
-precision).
+pass compute, plus the FP8 preparation (exact rotation, block quantisation
+decided in the kernel's fp32 precision).
 Only tests/, __graft_entry__.smoke() and bench.py's CPU baseline leg may import
 this package; the CUDA library and its binding never do, and this package never
 imports them.
