@@ -33,6 +33,7 @@ sys.path.insert(0, HERE)
 import workloads  # noqa: E402
 
 METRIC = "attention fwd TFLOPS (BF16 / FP8) and % of B200 tensor-core peak"
+METRIC_BWD = "attention bwd TFLOPS (BF16, 2.5x forward FLOPs) and % of B200 tensor-core peak"
 DEFAULT_WORKLOAD = "llm_train_causal"
 L2_BYTES = 126 * 1024 * 1024
 
@@ -46,6 +47,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the backward pass (attn_bwd) of a BF16 workload instead of the forward")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch size (small profiling captures only)")
     return ap.parse_args()
@@ -317,6 +320,69 @@ class Step:
         mark("attn_fwd_sm100")
 
 
+class BwdStep:
+    """One backward pass (attn_bwd: D_i, dK/dV, dQ) over resident inputs: Q, K, V,
+    dO and the forward's O and LSE (computed once, outside the timed region)."""
+
+    def __init__(self, lib, w, x, dev):
+        import torch
+        self.lib, self.w, self.dev = lib, w, dev
+        self.q, self.k, self.v = (x[n].to(dev) for n in ("q", "k", "v"))
+        g = torch.Generator().manual_seed(w.seed + 1)
+        self.dout = torch.randn((w.B, w.H, w.N, w.d), generator=g).to(torch.bfloat16).to(dev)
+        self.o, self.lse = lib.forward(self.q, self.k, self.v, causal=w.causal)
+        self.grads = [torch.empty_like(self.q) for _ in range(3)]
+        self.ws_bytes = lib.attn_bwd_workspace_bytes(w.B, w.H, w.N, w.d)
+        self.ws = torch.empty(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.copies = 1
+        self.launches = 3
+        self.kernels = ["attn_bwd"]
+
+    def run_device(self, stream, mark=None):
+        lib, w = self.lib, self.w
+        st = lib.attn_bwd(self.q.data_ptr(), self.k.data_ptr(), self.v.data_ptr(), self.o.data_ptr(),
+                          self.lse.data_ptr(), self.dout.data_ptr(), *(t.data_ptr() for t in self.grads),
+                          self.ws.data_ptr(), self.ws_bytes, w.B, w.H, w.N, w.d, w.scale, int(w.causal),
+                          stream.cuda_stream)
+        if st:
+            raise lib.AttnError(st, "attn_bwd")
+        if mark:
+            mark("attn_bwd")
+
+
+def time_e2e_bwd(lib, w, step, dev, stream, steps):
+    """The backward end to end through the public Python API: Q, K, V, O, LSE and
+    dO copied in from pinned host memory, dQ, dK, dV read back, every step."""
+    import torch
+    src = {"q": step.q, "k": step.k, "v": step.v, "o": step.o, "lse": step.lse, "dout": step.dout}
+    host = {n: t.cpu().pin_memory() for n, t in src.items()}
+    dev_in = {n: torch.empty_like(t) for n, t in src.items()}
+    outs_h = [torch.empty(step.q.shape, dtype=torch.bfloat16).pin_memory() for _ in range(3)]
+    outs_d = [torch.empty_like(step.q) for _ in range(3)]
+
+    def one():
+        with torch.cuda.stream(stream):
+            for n in src:
+                dev_in[n].copy_(host[n], non_blocking=True)
+            lib.backward(dev_in["q"], dev_in["k"], dev_in["v"], dev_in["o"], dev_in["lse"], dev_in["dout"],
+                         causal=w.causal, dq=outs_d[0], dk=outs_d[1], dv=outs_d[2], workspace=step.ws,
+                         stream=stream)
+            for h, d_ in zip(outs_h, outs_d):
+                h.copy_(d_, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs_h)
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
 def time_device(step, stream, steps, warmup, world, dev, clk=None):
     """Returns (ms for `steps` steps on this rank, {kernel: mean ms per launch}).
     Events are recorded on the launching stream before the loop and after every
@@ -464,6 +530,25 @@ def roofline(w, kern_ms, sm_mhz, workload):
     return roof
 
 
+def roofline_bwd(w, kern_ms, sm_mhz):
+    """Roofline of the backward pass as one unit (its three launches: D_i, dK/dV,
+    dQ), algorithmic FLOPs 2.5x the forward's, against the bf16 tensor-core peak."""
+    peak, _, peak_src = measured_peaks()
+    k_ms = kern_ms["attn_bwd"]
+    fl = 2.5 * w.flops
+    achieved = fl / (k_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": None, "peak_source": f"{peak_src} bf16 burst",
+            "kernel": "attn_bwd (attn_bwd_rowdot + attn_bwd_dkdv + attn_bwd_dq)", "algorithmic_flops": fl,
+            "kernel_ms": round(k_ms, 5), "datasheet_peak": DATASHEET_TFLOPS["bf16"],
+            "frac_of_datasheet_peak": round(achieved / DATASHEET_TFLOPS["bf16"], 4)}
+    hw = hw_peak_tflops("bf16", sm_mhz)
+    if hw:
+        roof["hw_peak_at_sampled_clock"] = round(hw, 1)
+        roof["frac_of_hw_peak_at_sampled_clock"] = round(achieved / hw, 4)
+    return roof
+
+
 def fp8_gemm_burst_tflops(dev, n=8192, reps=10):
     """Measured dense E4M3 GEMM rate (library GEMM, torch._scaled_mm, n^3, best of
     `reps`), the FP8 counterpart of the measured bf16 burst peak."""
@@ -505,7 +590,9 @@ def run_ours(args):
     if w.fp8:
         x["rot64"], x["rot"] = workloads.make_rotation(w.d, w.seed + 7919)
     stream = torch.cuda.Stream(dev)
-    step = Step(lib, w, x, dev)
+    if args.bwd and w.fp8:
+        raise SystemExit("--bwd needs a BF16 workload")
+    step = BwdStep(lib, w, x, dev) if args.bwd else Step(lib, w, x, dev)
     with ClockSampler(gpu_smi_id(dev, local)) as clk:
         ms_rank, kern_ms = time_device(step, stream, args.steps, max(3, args.warmup), world, dev, clk)
     st = lib.attn_get_device_status(stream.cuda_stream)
@@ -514,29 +601,36 @@ def run_ours(args):
     clocks = clk.summary()
     ms_total = max_over_ranks(ms_rank, world, dev)
     ms_step = ms_total / args.steps
-    flops_rank = w.flops
+    # the backward's 5 products (S, dP, dV, dK, dQ) against the forward's 2: 2.5x
+    flops_rank = w.flops * (2.5 if args.bwd else 1.0)
     tflops = flops_rank * world / (ms_step * 1e-3) / 1e12
     # e2e through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e_ms, h2d, d2h = time_e2e(lib, w, x, dev, stream, args.e2e_steps)
+        if args.bwd:
+            e2e_ms, h2d, d2h = time_e2e_bwd(lib, w, step, dev, stream, args.e2e_steps)
+        else:
+            e2e_ms, h2d, d2h = time_e2e(lib, w, x, dev, stream, args.e2e_steps)
         e2e_ms = max_over_ranks(e2e_ms, world, dev)
         e2e = {"value": round(flops_rank * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
     dt = "fp8" if w.fp8 else "bf16"
-    roof = roofline(w, kern_ms, clocks.get("sm_mhz"), args.workload)
+    roof = (roofline_bwd(w, kern_ms, clocks.get("sm_mhz")) if args.bwd
+            else roofline(w, kern_ms, clocks.get("sm_mhz"), args.workload))
     if w.fp8:
         roof["measured_fp8_gemm_burst_tflops"] = fp8_gemm_burst_tflops(dev)
     cpu = None
     if rank == 0 and world == 1:
-        cpu = cpu_baseline(w, budget_s=float(os.environ.get("ATTN_CPU_BASELINE_S", "15")))
+        budget = float(os.environ.get("ATTN_CPU_BASELINE_S", "15"))
+        cpu = cpu_baseline_bwd(w, budget) if args.bwd else cpu_baseline(w, budget_s=budget)
     mhz = clocks.get("sm_mhz")
     line = {
-        "metric": METRIC, "value": round(tflops, 3), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "metric": METRIC_BWD if args.bwd else METRIC, "value": round(tflops, 3), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if w.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B * world, "B_per_gpu": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "causal": w.causal, "flops_per_step_per_gpu": w.flops,
+                   "causal": w.causal, "flops_per_step_per_gpu": flops_rank,
+                   "pass": "backward" if args.bwd else "forward",
                    "parallelism": f"replicas x{world} (independent (b,h) units, no collective)",
                    "l2": "inputs larger than L2 (no flush)" if step.copies == 1 else
                    f"inputs smaller than L2: the timed loop rotates through {step.copies} copies "
@@ -611,6 +705,27 @@ def cpu_baseline(w, budget_s=15.0):
     dt = (time.perf_counter() - t0) / reps
     return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
             "sample": desc + f", fp64 numpy, {reps} repetitions"}
+
+
+def cpu_baseline_bwd(w, budget_s=15.0):
+    """The backward oracle as it stands on the host cores, one head of the workload
+    in full (its algorithmic FLOPs: 2.5x the head's forward FLOPs)."""
+    import torch
+    from oracle import attention_bwd_fp64
+    gen = torch.Generator().manual_seed(777)
+    q, k, v, do = (torch.randn((1, 1, w.N, w.d), generator=gen).to(torch.bfloat16).double().numpy()
+                   for _ in range(4))
+    fl = 2.5 * w.flops / (w.B * w.H)
+    t0 = time.perf_counter()
+    attention_bwd_fp64(q, k, v, do, w.scale, w.causal)
+    one = time.perf_counter() - t0
+    reps = max(1, int(budget_s / max(one, 1e-3)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        attention_bwd_fp64(q, k, v, do, w.scale, w.causal)
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(fl / dt / 1e12, 6), "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"1 head of {w.name} in full (N={w.N}, d={w.d}), fp64 numpy backward, {reps} repetitions"}
 
 
 def run_reference(args):

@@ -30,6 +30,8 @@ SIGNATURES = {
     "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_fwd_inject_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, ctypes.c_ulonglong, _P]),
+    "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_abi_version": (_I, []),
 }
@@ -67,6 +69,15 @@ def attn_quantize_fp8(x, rot, x8, scales, B, H, N, d, stream):
 
 def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, scale, causal, stream):
     return load().attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, scale, causal, stream)
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, scale, causal, stream):
+    return load().attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, scale,
+                           causal, stream)
+
+
+def attn_bwd_workspace_bytes(B, H, N, d):
+    return load().attn_bwd_workspace_bytes(B, H, N, d)
 
 
 def attn_fwd_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit, wait_limit_cycles, stream):
@@ -196,6 +207,38 @@ def forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale=None,
            "attn_fwd_fp8")
     _check_device(check, sp, "attn_fwd_fp8")
     return out, lse
+
+
+def backward(q, k, v, o, lse, dout, causal=False, scale=None, dq=None, dk=None, dv=None, workspace=None,
+             stream=None, check=False):
+    """dQ, dK, dV of attention for bf16 CUDA tensors [B, H, N, d], given the
+    forward's O and LSE and dout = dL/dO. The workspace (D_i per row) is
+    allocated with torch unless given. Asynchronous like forward()."""
+    import torch
+    B, H, N, d = _shape4(q)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _expect(t, name, (B, H, N, d), torch.bfloat16, q.device)
+    _expect(lse, "lse", (B, H, N), torch.float32, q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _expect(t, name, (B, H, N, d), torch.bfloat16, q.device)
+    need = attn_bwd_workspace_bytes(B, H, N, d)
+    if need == 0:
+        raise AttnError(ATTN_ERR_UNSUPPORTED, "attn_bwd_workspace_bytes")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if not workspace.is_cuda or workspace.device != q.device or workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace must be a CUDA buffer of at least {need} bytes on {q.device}")
+    sc = 0.0 if scale is None else float(scale)
+    sp = _stream_ptr(q, stream)
+    _check(attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), dout.data_ptr(),
+                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                    workspace.numel() * workspace.element_size(), B, H, N, d, sc, int(bool(causal)), sp),
+           "attn_bwd")
+    _check_device(check, sp, "attn_bwd")
+    return dq, dk, dv
 
 
 def flops(B, H, N, d, causal):

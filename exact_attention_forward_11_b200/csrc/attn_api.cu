@@ -13,6 +13,7 @@
 
 #include "attn_b200.h"
 #include "attn_b200_testing.h"
+#include "attn_bwd_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
 #include "fp8_prep_kernel.cuh"
 
@@ -75,11 +76,11 @@ int sm_count() {
 // belongs to the function on the current device; later calls skip the driver
 // call). `tag` identifies the kernel. A failed launch forgets the flag, so a
 // context that was reset gets the attribute again on the next call.
-std::atomic<uint32_t> g_smem_done[64][8];
+std::atomic<uint32_t> g_smem_done[64][16];
 
 void forget_smem(int tag) {
   int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && tag < 8)
+  if (cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < 64 && tag < 16)
     g_smem_done[dev][tag].store(0u, std::memory_order_release);
 }
 
@@ -87,9 +88,9 @@ bool set_smem_once(const void* func, int bytes, int tag) {
   auto& done = g_smem_done;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return false;
-  if (dev < 64 && tag < 8 && done[dev][tag].load(std::memory_order_acquire)) return true;
+  if (dev < 64 && tag < 16 && done[dev][tag].load(std::memory_order_acquire)) return true;
   if (cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
-  if (dev < 64 && tag < 8) done[dev][tag].store(1u, std::memory_order_release);
+  if (dev < 64 && tag < 16) done[dev][tag].store(1u, std::memory_order_release);
   return true;
 }
 
@@ -164,6 +165,52 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   }
   return ATTN_OK;
 }
+
+template <int D>
+attn_status launch_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* dout, void* dq, void* dk, void* dv, float* dd, int BH, int N, float scale,
+                       int causal, cudaStream_t stream) {
+  using C = attn::BwdCfg<D>;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!encode_qkv_map(&tq, q, false, D, N, BH, 128) || !encode_qkv_map(&tk, k, false, D, N, BH, 128) ||
+      !encode_qkv_map(&tv, v, false, D, N, BH, 128) || !encode_qkv_map(&tdo, dout, false, D, N, BH, 128))
+    return ATTN_ERR_CUDA;
+  auto kdkdv = attn::attn_bwd_dkdv<C>;
+  auto kdq = attn::attn_bwd_dq<C>;
+  const int tag = D == 128 ? 5 : 6;
+  if (!set_smem_once(reinterpret_cast<const void*>(kdkdv), C::DKDV_SMEM, tag) ||
+      !set_smem_once(reinterpret_cast<const void*>(kdq), C::DQ_SMEM, tag + 2))
+    return ATTN_ERR_CUDA;
+  // D_i = dO_i . O_i (D/8 lanes per row)
+  const long long rows = static_cast<long long>(BH) * N;
+  const long long threads = rows * (D / 8);
+  attn::attn_bwd_rowdot<D><<<static_cast<unsigned>((threads + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), dd, rows);
+  attn::BwdParams p;
+  p.N = N;
+  p.BH = BH;
+  p.causal = causal;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.lse = lse;
+  p.dd = dd;
+  p.dq = static_cast<__nv_bfloat16*>(dq);
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.timeout_cycles = kWaitLimitCycles;
+  const int QB = (N + 127) / 128;
+  kdkdv<<<QB * BH, C::THREADS, C::DKDV_SMEM, stream>>>(tq, tk, tv, tdo, p);
+  kdq<<<QB * BH, C::THREADS, C::DQ_SMEM, stream>>>(tq, tk, tv, tdo, p);
+  if (cudaGetLastError() != cudaSuccess) {
+    forget_smem(tag);
+    forget_smem(tag + 2);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+// Bytes of workspace attn_bwd needs: D_i for every row, fp32, rounded to 256.
+size_t bwd_workspace_bytes(long long BH, long long N) { return static_cast<size_t>((BH * N * 4 + 255) / 256 * 256); }
 
 }  // namespace
 
@@ -268,6 +315,31 @@ attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* s
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  return bwd_workspace_bytes(static_cast<long long>(B) * H, N);
+}
+
+attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                     void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int B, int H, int N,
+                     int d, float scale, int causal, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr || dout == nullptr ||
+      dq == nullptr || dk == nullptr || dv == nullptr || workspace == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = resolve_scale(scale, d); s != ATTN_OK) return s;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (workspace_bytes < bwd_workspace_bytes(static_cast<long long>(B) * H, N)) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned16(workspace))
+    return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* dd = static_cast<float*>(workspace);
+  if (d == 128) return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, dd, B * H, N, scale, causal, st);
+  return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, dd, B * H, N, scale, causal, st);
 }
 
 attn_status attn_get_device_status(void* stream) {

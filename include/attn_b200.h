@@ -1,6 +1,6 @@
 /*
- * attn_b200.h - C ABI of a fused scaled-dot-product attention forward for
- * NVIDIA B200 (sm_100a).
+ * attn_b200.h - C ABI of a fused scaled-dot-product attention forward (and
+ * its backward pass) for NVIDIA B200 (sm_100a).
  *
  * The operation ("Self-Attention, CUDA kernels and FlashAttention", section 1,
  * eq. Scores and eq. Attention; section 3, tiling / online-softmax / recompute
@@ -43,6 +43,8 @@
 #else
 #define ATTN_API
 #endif
+
+#include <stddef.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -120,6 +122,40 @@ ATTN_API attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8
                          const float* q_scale, const float* k_scale, const float* v_scale,
                          void* o, float* lse, int B, int H, int N, int d, float scale,
                          int causal, void* stream);
+
+/*
+ * attn_bwd - backward pass of attn_fwd (BF16) from the saved statistic LSE
+ * ("Self-Attention, CUDA kernels and FlashAttention", section 3, recompute
+ * bullet: the forward keeps only the per-row normalisation statistics, and the
+ * backward recomputes the attention weights tile by tile in on-chip memory
+ * instead of reading a stored N x N matrix). For dL/dO = dout it computes
+ *     P  = exp(scale Q K^T - LSE)   (causal: 0 for key j > query i)
+ *     dV = P^T dO,   dP = dO V^T,   D_i = sum_c dO_ic O_ic,
+ *     dS = P * (dP - D),   dQ = scale dS K,   dK = scale dS^T Q.
+ *   q, k, v    : [B, H, N, d] bf16, the forward's inputs.
+ *   o, lse     : the forward's outputs for those inputs ([B, H, N, d] bf16 and
+ *                [B, H, N] fp32, natural log), as attn_fwd wrote them.
+ *   dout       : [B, H, N, d] bf16 gradient of the loss with respect to O.
+ *   dq, dk, dv : [B, H, N, d] bf16 outputs (must not alias the inputs).
+ *   workspace  : device scratch of at least attn_bwd_workspace_bytes(B, H, N, d)
+ *                bytes, 16-byte aligned, owned by the caller; it holds D_i and
+ *                is overwritten. Calls that overlap on the GPU need separate
+ *                workspaces.
+ *   scale, causal: the values the forward used (scale == 0: 1/sqrt(d)).
+ *   d          : 64 or 128 (else ATTN_ERR_UNSUPPORTED).
+ * LSE is taken as the saved statistic, not a differentiated output: no gradient
+ * flows into it. Three kernels run on `stream` in order (D_i, then dK and dV,
+ * then dQ); nothing is allocated. Errors as for attn_fwd, plus
+ * ATTN_ERR_INVALID_ARG for a null workspace or one smaller than required.
+ */
+ATTN_API attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                     size_t workspace_bytes, int B, int H, int N, int d, float scale, int causal,
+                     void* stream);
+
+/* attn_bwd_workspace_bytes - workspace attn_bwd needs for this shape (0 for an
+ * invalid or unsupported shape). Host only; launches nothing. */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
 
 /*
  * attn_get_device_status - synchronises `stream`, then reads and clears the

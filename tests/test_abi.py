@@ -106,3 +106,26 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(m, "_lib", None)
     with pytest.raises(RuntimeError, match="not built"):
         m.load()
+
+
+def test_bwd_argument_validation(lib):
+    f = lib.attn_bwd
+    need = lib.attn_bwd_workspace_bytes(1, 2, 100, 128)
+    assert need == 1024                       # 2 x 100 rows x 4 bytes, rounded up to 256
+    assert lib.attn_bwd_workspace_bytes(1, 1, 8, 96) == 0
+    assert lib.attn_bwd_workspace_bytes(0, 1, 8, 128) == 0
+    ok = [FAKE] * 10 + [need, 1, 2, 100, 128, 0.0, 0, None]
+
+    def call(i=None, val=None):
+        a = list(ok)
+        if i is not None:
+            a[i] = val
+        return f(*a)
+    assert call(9, None) == lib.ATTN_ERR_INVALID_ARG           # no workspace
+    assert call(10, need - 4) == lib.ATTN_ERR_INVALID_ARG      # workspace too small
+    assert call(4, None) == lib.ATTN_ERR_INVALID_ARG           # no lse
+    assert call(16, 3) == lib.ATTN_ERR_INVALID_ARG             # causal flag
+    assert call(15, -1.0) == lib.ATTN_ERR_INVALID_ARG          # negative scale
+    assert call(14, 96) == lib.ATTN_ERR_UNSUPPORTED
+    assert call(6, FAKE + 8) == lib.ATTN_ERR_MISALIGNED
+    assert call(9, FAKE + 4) == lib.ATTN_ERR_MISALIGNED
