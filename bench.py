@@ -34,6 +34,7 @@ import workloads  # noqa: E402
 
 METRIC = "attention fwd TFLOPS (BF16 / FP8) and % of B200 tensor-core peak"
 METRIC_BWD = "attention bwd TFLOPS (BF16, 2.5x forward FLOPs) and % of B200 tensor-core peak"
+METRIC_W4A16 = "W4A16 GEMM TFLOPS (fp16 activations, int4 weights dequantised on the fly) and % of HBM roofline"
 DEFAULT_WORKLOAD = "llm_train_causal"
 L2_BYTES = 126 * 1024 * 1024
 
@@ -43,7 +44,8 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=sorted(workloads.WORKLOADS) + sorted(workloads.GEMM_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
@@ -383,6 +385,111 @@ def time_e2e_bwd(lib, w, step, dev, stream, steps):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
+class GemmStep:
+    """One W4A16 GEMM launch over resident operands. The weights (117 MB for the
+    decode workload) are larger than L2, so every step streams them from HBM."""
+
+    def __init__(self, lib, wl, dev, seed):
+        import torch
+        self.lib, self.wl = lib, wl
+        x, qw, s, z = workloads.make_w4a16(wl.M, wl.N, wl.K, seed)
+        self.host = (x, qw, s, z)
+        self.x, self.qw, self.s, self.z = (t.to(dev) for t in (x, qw, s, z))
+        self.y = torch.empty((wl.M, wl.N), dtype=torch.float16, device=dev)
+        self.copies = 1
+        self.launches = 1
+        self.kernels = ["w4a16_gemm_sm100"]
+
+    def bytes(self):
+        wl = self.wl
+        return (wl.K * wl.N // 2 + (wl.K // 128) * wl.N * 3 + wl.M * wl.K * 2 + wl.M * wl.N * 2)
+
+    def run_device(self, stream, mark=None):
+        wl, lib = self.wl, self.lib
+        st = lib.w4a16_gemm(self.x.data_ptr(), self.qw.data_ptr(), self.s.data_ptr(), self.z.data_ptr(),
+                            self.y.data_ptr(), wl.M, wl.N, wl.K, stream.cuda_stream)
+        if st:
+            raise lib.AttnError(st, "w4a16_gemm")
+        if mark:
+            mark("w4a16_gemm_sm100")
+
+
+def run_gemm(args, lib, dev, rank, world, local):
+    """Bench line of a W4A16 GEMM workload (HBM roofline on the algorithmic bytes:
+    packed weights, scales, zero points, X read once, Y written once)."""
+    import torch
+    wl = workloads.GEMM_WORKLOADS[args.workload]
+    stream = torch.cuda.Stream(dev)
+    step = GemmStep(lib, wl, dev, wl.seed + 7919 * rank)
+    with ClockSampler(gpu_smi_id(dev, local)) as clk:
+        ms_rank, kern_ms = time_device(step, stream, args.steps, max(3, args.warmup), world, dev, clk)
+    st = lib.attn_get_device_status(stream.cuda_stream)
+    if st != lib.ATTN_OK:
+        raise lib.AttnError(st, "device status")
+    clocks = clk.summary()
+    ms_step = max_over_ranks(ms_rank, world, dev) / args.steps
+    tflops = wl.flops * world / (ms_step * 1e-3) / 1e12
+    _, hbm, peak_src = measured_peaks()
+    k_ms = kern_ms["w4a16_gemm_sm100"]
+    nbytes = step.bytes()
+    gbs = nbytes / (k_ms * 1e-3) / 1e9
+    roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s", "frac": round(gbs / hbm, 4),
+            "traffic": None, "peak_source": f"{peak_src} copy bandwidth", "kernel": "w4a16_gemm_sm100",
+            "algorithmic_bytes": nbytes, "kernel_ms": round(k_ms, 5)}
+    e2e = None
+    if not args.no_e2e:
+        host = [t.pin_memory() for t in step.host]
+        dev_t = [torch.empty_like(t, device=dev) for t in host]
+        y_h = torch.empty((wl.M, wl.N), dtype=torch.float16).pin_memory()
+
+        def one():
+            with torch.cuda.stream(stream):
+                for h, d_ in zip(host, dev_t):
+                    d_.copy_(h, non_blocking=True)
+                lib.w4a16_matmul(*dev_t, out=step.y, stream=stream)
+                y_h.copy_(step.y, non_blocking=True)
+        one()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, world, dev)
+        e2e = {"value": round(wl.flops * world / (e_ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host),
+               "d2h_bytes_per_step": y_h.numel() * 2, "ms_per_step": round(e_ms, 4)}
+    cpu = cpu_baseline_gemm(wl) if rank == 0 and world == 1 else None
+    mhz = clocks.get("sm_mhz")
+    return {
+        "metric": METRIC_W4A16, "value": round(tflops, 3), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16xint4", "data": "synthetic",
+        "config": {"workload": wl.name, "M": wl.M, "N": wl.N, "K": wl.K, "group": 128,
+                   "parallelism": f"replicas x{world}", "l2": "weights larger than L2 (no flush)"},
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": args.steps,
+        "kernel_ms": {k: round(v, 5) for k, v in kern_ms.items()},
+        "cycles_per_step": None if mhz is None else round(ms_step * 1e-3 * mhz * 1e6), "clocks": clocks}
+
+
+def cpu_baseline_gemm(wl, budget_s=10.0):
+    """The W4A16 oracle as it stands, on 512 of the N output columns."""
+    from oracle.w4a16 import w4a16_gemm_fp64
+    x, qw, s, z = workloads.make_w4a16(wl.M, 512, wl.K, 99)
+    args = (x.numpy(), qw.numpy(), s.numpy(), z.numpy())
+    t0 = time.perf_counter()
+    w4a16_gemm_fp64(*args)
+    one = time.perf_counter() - t0
+    reps = max(1, int(budget_s / max(one, 1e-3)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        w4a16_gemm_fp64(*args)
+    dt = (time.perf_counter() - t0) / reps
+    return {"value": round(2.0 * wl.M * 512 * wl.K / dt / 1e12, 6), "unit": "TFLOPS", "cores": blas_threads(),
+            "kind": "oracle", "sample": f"{wl.M} x 512 x {wl.K} (512 of {wl.N} columns), {reps} repetitions"}
+
+
 def time_device(step, stream, steps, warmup, world, dev, clk=None):
     """Returns (ms for `steps` steps on this rank, {kernel: mean ms per launch}).
     Events are recorded on the launching stream before the loop and after every
@@ -581,6 +688,14 @@ def run_ours(args):
     init_dist("nccl", world)
     import exact_attention_forward_11_b200 as lib
     lib.load()
+    if args.workload in workloads.GEMM_WORKLOADS:
+        line = run_gemm(args, lib, dev, rank, world, local)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     w = workloads.WORKLOADS[args.workload]
     if args.batch is not None:
         import dataclasses
@@ -732,10 +847,36 @@ def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    w = workloads.WORKLOADS[args.workload]
-    # each step: one head x 64 query rows of the workload (bounded so that
-    # warm-up + K steps finish within minutes)
-    call, fl, desc = oracle_sample(w, 64, 1, 4321)
+    if args.workload in workloads.GEMM_WORKLOADS:
+        # each step: the W4A16 oracle on 128 of the N output columns
+        wl = workloads.GEMM_WORKLOADS[args.workload]
+        from oracle.w4a16 import w4a16_gemm_fp64
+        ops = [t.numpy() for t in workloads.make_w4a16(wl.M, 128, wl.K, 4321)]
+
+        def call():
+            return w4a16_gemm_fp64(*ops)
+        fl, desc, metric = 2.0 * wl.M * 128 * wl.K, f"{wl.M} x 128 x {wl.K} of {wl.name}", METRIC_W4A16
+        cfg = {"workload": wl.name, "M": wl.M, "N": wl.N, "K": wl.K}
+    elif args.bwd:
+        # each step: the backward oracle on one head of the workload, N capped at 1024 rows
+        w = workloads.WORKLOADS[args.workload]
+        from oracle import attention_bwd_fp64
+        n = min(w.N, 1024)
+        gen = __import__("torch").Generator().manual_seed(4321)
+        ops = [__import__("torch").randn((1, 1, n, w.d), generator=gen).double().numpy() for _ in range(4)]
+
+        def call():
+            return attention_bwd_fp64(*ops, w.scale, w.causal)
+        fl = 2.5 * 4.0 * n * n * w.d / (2 if w.causal else 1)
+        desc, metric = f"1 head of {w.name} with N = {n}", METRIC_BWD
+        cfg = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal, "pass": "backward"}
+    else:
+        w = workloads.WORKLOADS[args.workload]
+        # each step: one head x 64 query rows of the workload (bounded so that
+        # warm-up + K steps finish within minutes)
+        call, fl, desc = oracle_sample(w, 64, 1, 4321)
+        metric = METRIC
+        cfg = {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal}
     for _ in range(max(1, args.warmup)):
         call()
     t0 = time.perf_counter()
@@ -743,11 +884,10 @@ def run_reference(args):
         call()
     dt = (time.perf_counter() - t0) / args.steps
     v = fl / dt / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": round(v, 6), "unit": "TFLOPS", "n_gpus": world,
+    line = {"impl": "reference", "metric": metric, "value": round(v, 6), "unit": "TFLOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal},
+            "dtype": "f64", "data": "synthetic", "config": cfg,
             "cpu_baseline": {"value": round(v, 6), "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
                              "sample": desc + " per step"},
             "e2e": {"value": round(v, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -32,6 +32,7 @@ SIGNATURES = {
     "attn_fwd_inject_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, ctypes.c_ulonglong, _P]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "w4a16_gemm": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_abi_version": (_I, []),
 }
@@ -78,6 +79,10 @@ def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H
 
 def attn_bwd_workspace_bytes(B, H, N, d):
     return load().attn_bwd_workspace_bytes(B, H, N, d)
+
+
+def w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream):
+    return load().w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream)
 
 
 def attn_fwd_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit, wait_limit_cycles, stream):
@@ -239,6 +244,28 @@ def backward(q, k, v, o, lse, dout, causal=False, scale=None, dq=None, dk=None, 
            "attn_bwd")
     _check_device(check, sp, "attn_bwd")
     return dq, dk, dv
+
+
+def w4a16_matmul(x, qweight, scales, zeros, out=None, stream=None, check=False):
+    """Y = X W for fp16 X [M, K] and W given as packed int4 (int32 [K/8, N]), fp16
+    scales [K/128, N] and uint8 zero points [K/128, N] (include/w4a16_b200.h)."""
+    import torch
+    if x.dim() != 2:
+        raise ValueError("x must be [M, K]")
+    M, K = x.shape
+    _expect(x, "x", (M, K), torch.float16, x.device)
+    N = qweight.shape[1] if qweight.dim() == 2 else -1
+    _expect(qweight, "qweight", (K // 8, N), torch.int32, x.device)
+    _expect(scales, "scales", (K // 128, N), torch.float16, x.device)
+    _expect(zeros, "zeros", (K // 128, N), torch.uint8, x.device)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float16, device=x.device)
+    _expect(out, "out", (M, N), torch.float16, x.device)
+    sp = _stream_ptr(x, stream)
+    _check(w4a16_gemm(x.data_ptr(), qweight.data_ptr(), scales.data_ptr(), zeros.data_ptr(), out.data_ptr(),
+                      M, N, K, sp), "w4a16_gemm")
+    _check_device(check, sp, "w4a16_gemm")
+    return out
 
 
 def flops(B, H, N, d, causal):

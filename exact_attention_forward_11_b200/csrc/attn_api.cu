@@ -13,9 +13,11 @@
 
 #include "attn_b200.h"
 #include "attn_b200_testing.h"
+#include "w4a16_b200.h"
 #include "attn_bwd_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
 #include "fp8_prep_kernel.cuh"
+#include "w4a16_kernel.cuh"
 
 namespace {
 
@@ -58,6 +60,21 @@ bool encode_qkv_map(CUtensorMap* map, const void* base, bool fp8, int d, int N, 
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// Map over a row-major matrix [outer, inner] viewed as {inner, outer, 1}, box
+// {box_inner, box_outer, 1}: elements past the matrix read as zero.
+bool encode_matrix_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int elem, long long inner,
+                       long long outer, int box_inner, int box_outer, bool swizzle128) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(outer), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * elem, static_cast<cuuint64_t>(inner) * elem * outer};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_outer), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Number of SMs of the current device (cached per device ordinal).
@@ -340,6 +357,41 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   float* dd = static_cast<float*>(workspace);
   if (d == 128) return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, dd, B * H, N, scale, causal, st);
   return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, dd, B * H, N, scale, causal, st);
+}
+
+attn_status w4a16_gemm(const void* x, const void* qweight, const void* scales, const void* zeros, void* y, int M,
+                       int N, int K, void* stream) {
+  using C = attn::W4Cfg;
+  if (x == nullptr || qweight == nullptr || scales == nullptr || zeros == nullptr || y == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (M < 1 || N < 1 || K < 1) return ATTN_ERR_INVALID_ARG;
+  if (M > C::MAX_M || N % C::BN != 0 || K % C::GROUP != 0) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y))
+    return ATTN_ERR_MISALIGNED;
+  if (static_cast<long long>(K) * N >= (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  const int mpad = (M + 15) / 16 * 16;
+  CUtensorMap tx, tw, ts, tz;
+  if (!encode_matrix_map(&tx, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, 64, mpad, true) ||
+      !encode_matrix_map(&tw, qweight, CU_TENSOR_MAP_DATA_TYPE_INT32, 4, N, K / 8, C::BN, 16, false) ||
+      !encode_matrix_map(&ts, scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, N, K / C::GROUP, C::BN, 1, false) ||
+      !encode_matrix_map(&tz, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / C::GROUP, C::BN, 1, false))
+    return ATTN_ERR_CUDA;
+  const int smem = C::smem_bytes(mpad);
+  if (!set_smem_once(reinterpret_cast<const void*>(attn::w4a16_gemm_sm100), C::smem_bytes(C::MAX_M), 9))
+    return ATTN_ERR_CUDA;
+  attn::W4Params p;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.mpad = mpad;
+  p.y = static_cast<__half*>(y);
+  p.timeout_cycles = kWaitLimitCycles;
+  attn::w4a16_gemm_sm100<<<N / C::BN, C::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(tx, tw, ts, tz, p);
+  if (cudaGetLastError() != cudaSuccess) {
+    forget_smem(9);
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
 }
 
 attn_status attn_get_device_status(void* stream) {

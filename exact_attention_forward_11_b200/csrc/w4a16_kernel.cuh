@@ -1,0 +1,245 @@
+// w4a16_kernel.cuh - GEMM with 4-bit weights dequantised on the fly (W4A16).
+//
+// "FlashAttention scaling, multi-GPU training and weight quantization", section 3,
+// the W4A16 kernels paragraph: the packed 4-bit weights (eight to a 32-bit word)
+// are read from HBM, unpacked in registers with shifts and masks, turned into
+// 16-bit floats with the stored scale and zero point, and fed to the tensor cores
+// with the 16-bit activations; the expanded weights never go back to memory.
+//
+//   Y[M, N] = X[M, K] W[K, N],  W[k, n] = fp16((q[k, n] - z[g, n]) * s[g, n]),
+//   g = k / 128, q from qweight[k / 8, n] (weight 8w + PERM[i] in bits 4i..4i+3,
+//   PERM = 0 2 4 6 1 3 5 7), fp32 accumulation, Y rounded to fp16.
+//
+// Decode-sized M (1..128 tokens) makes the GEMM HBM-bound on the weights (half a
+// byte per weight), so the layout is chosen for a stream: one CTA per 128 output
+// columns walks K in 128-deep slices. The MMA is issued with the operands swapped
+// (D[128 columns n][M tokens] = W^T X^T) so that M = 128 is the weight side and
+// the token count only sets the MMA's N (padded to a multiple of 16). The
+// dequantised weights go straight from registers into tensor memory (one thread
+// per output column = one TMEM lane, tcgen05.st) and are the MMA's A operand
+// from TMEM; only the small X slice is read from shared memory by the MMA.
+//
+// CTA: 8 warps. warp 0 TMA producer (weight words, scales, zero points and the X
+// slice of each K slice into a 4-stage ring), warp 1 MMA issuer (owns TMEM),
+// warps 2-3 idle, warps 4-7 dequantise (thread t: column n0 + t) and write Y.
+// TMEM: two 64-column A buffers (a 128-deep slice of fp16 pairs) and the
+// MPAD-column fp32 accumulator. Every wait is bounded (Waiter).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "sm100.cuh"
+#include "status.cuh"
+
+namespace attn {
+
+struct W4Cfg {
+  static constexpr int THREADS = 256;
+  static constexpr int NST = 4;
+  static constexpr int GROUP = 128;            // k per scale / zero point = k per slice
+  static constexpr int BN = 128;               // output columns per CTA
+  static constexpr int WQ_BYTES = 16 * BN * 4; // 16 words (128 k) x 128 columns
+  static constexpr int S_BYTES = BN * 2;
+  static constexpr int Z_BYTES = BN;
+  static constexpr int MAX_M = 128;
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr uint32_t T_A = 0;           // A buffers: [0, 64), [64, 128)
+  static constexpr uint32_t T_D = 128;         // accumulator: MPAD columns
+  // stage layout (offsets inside a stage; X first so its chunks stay 1024-aligned)
+  __host__ __device__ static constexpr int x_chunk(int mpad) { return mpad * 128; }
+  __host__ __device__ static constexpr int stage_bytes(int mpad) {
+    return ((2 * x_chunk(mpad) + WQ_BYTES + S_BYTES + Z_BYTES) + 1023) / 1024 * 1024;
+  }
+  __host__ __device__ static constexpr int bar_offset(int mpad) { return NST * stage_bytes(mpad); }
+  __host__ __device__ static constexpr int smem_bytes(int mpad) { return bar_offset(mpad) + 16 * 8 + 16 + 1024; }
+};
+
+struct W4Params {
+  int M, N, K;
+  int mpad;                  // M rounded up to a multiple of 16
+  __half* y;                 // [M, N]
+  uint64_t timeout_cycles;
+};
+
+__global__ void __launch_bounds__(W4Cfg::THREADS, 1)
+    w4a16_gemm_sm100(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                     const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z,
+                     const W4Params p) {
+  using namespace b200;
+  using C = W4Cfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int mpad = p.mpad;
+  const int SB = C::stage_bytes(mpad);
+  const int XC = C::x_chunk(mpad);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::bar_offset(mpad));
+  uint64_t* full = bars;                     // NST: TMA bytes
+  uint64_t* empty = full + C::NST;           // NST: MMA commit (X read) + 4 dequant warps (words read)
+  uint64_t* a_full = empty + C::NST;         // 2: 4 dequant warps
+  uint64_t* a_empty = a_full + 2;            // 2: MMA commit
+  uint64_t* done = a_empty + 2;              // 1
+  uint64_t* drain_bar = done + 1;            // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint32_t* abort_word = tmem_slot + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * C::BN;
+  const int G = p.K / C::GROUP;              // slices
+
+  auto x_at = [&](int s) { return smem + s * SB; };
+  auto w_at = [&](int s) { return reinterpret_cast<const uint32_t*>(smem + s * SB + 2 * XC); };
+  auto s_at = [&](int s) { return reinterpret_cast<const __half*>(smem + s * SB + 2 * XC + C::WQ_BYTES); };
+  auto z_at = [&](int s) { return smem + s * SB + 2 * XC + C::WQ_BYTES + C::S_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::NST; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 5);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(a_full + b, 4);
+      mbar_init(a_empty + b, 1);
+    }
+    mbar_init(done, 1);
+    mbar_init(drain_bar, 1);
+    *abort_word = 0u;
+    fence_barrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const Waiter waiter{abort_word, p.timeout_cycles};
+  auto wait_all = [&](uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, waiter.wait(bar, parity)); };
+  bool ok = true;
+
+  if (warp == 0) {
+    // ======================= producer =======================
+    if (elect_one()) {
+      tma_prefetch_desc(&tm_x);
+      tma_prefetch_desc(&tm_w);
+      tma_prefetch_desc(&tm_s);
+      tma_prefetch_desc(&tm_z);
+    }
+    __syncwarp();
+    const uint64_t pol_w = l2_policy_evict_first();   // weights are read once
+    const uint64_t pol_x = l2_policy_evict_last();    // X is read by every CTA
+    const uint32_t bytes = static_cast<uint32_t>(2 * XC + C::WQ_BYTES + C::S_BYTES + C::Z_BYTES);
+    int g = 0;
+    for (; g < G; ++g) {
+      const int s = g % C::NST;
+      if (g >= C::NST && !(ok = wait_all(empty + s, ((g / C::NST) - 1) & 1))) break;
+      if (elect_one()) {
+        mbar_arrive_expect_tx(full + s, bytes);
+        tma_load_3d(x_at(s), &tm_x, full + s, g * C::GROUP, 0, 0, pol_x);
+        tma_load_3d(x_at(s) + XC, &tm_x, full + s, g * C::GROUP + 64, 0, 0, pol_x);
+        tma_load_3d(const_cast<uint32_t*>(w_at(s)), &tm_w, full + s, n0, g * 16, 0, pol_w);
+        tma_load_3d(const_cast<__half*>(s_at(s)), &tm_s, full + s, n0, g, 0, pol_w);
+        tma_load_3d(z_at(s), &tm_z, full + s, n0, g, 0, pol_w);
+      }
+      __syncwarp();
+    }
+    if (!ok) {
+      if (lane == 0) record_timeout();
+      const uint64_t t0 = sm_clock();
+      for (int j = (g > C::NST ? g - C::NST : 0); j < g; ++j)
+        while (!mbar_try_wait(full + (j % C::NST), (j / C::NST) & 1) && sm_clock() - t0 < p.timeout_cycles) {
+        }
+    }
+  } else if (warp == 1) {
+    // ======================= MMA issuer =======================
+    const uint32_t leader = elect_one() ? 1u : 0u;
+    const uint32_t idesc = instr_desc(0u /* f16 */, 128, static_cast<uint32_t>(mpad), 0, 0);
+    constexpr uint32_t hi = smem_desc_hi(1024);
+    const uint32_t x_lo = smem_desc_lo(smem_addr(smem), 16);
+    for (int g = 0; g < G; ++g) {
+      const int s = g % C::NST, b = g & 1;
+      if (!(ok = wait_all(full + s, (g / C::NST) & 1))) break;
+      if (!(ok = wait_all(a_full + b, (g >> 1) & 1))) break;
+      tc_fence_after();
+      const uint32_t xa = x_lo + ((s * SB) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = ((kk >> 2) * XC + (kk & 3) * 32) >> 4;
+        mma_f16_ts(tmem_base + C::T_D, tmem_base + C::T_A + 64 * b + 8 * kk, smem_desc(xa + off, hi), idesc,
+                   (g > 0 || kk > 0) ? 1u : 0u, leader);
+      }
+      mma_commit(empty + s, leader);
+      mma_commit(a_empty + b, leader);
+    }
+    if (ok) mma_commit(done, leader);
+    if (!ok && lane == 0) record_timeout();
+    mma_commit(drain_bar, leader);
+    const uint64_t t0 = sm_clock();
+    while (!mbar_try_wait(drain_bar, 0) && sm_clock() - t0 < p.timeout_cycles) {
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ======================= dequantise, then Y =======================
+    const int wq = warp - 4;
+    const int t = wq * 32 + lane;                    // output column n0 + t, TMEM lane t
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    for (int g = 0; g < G; ++g) {
+      const int s = g % C::NST, b = g & 1;
+      if (!(ok = wait_all(full + s, (g / C::NST) & 1))) break;
+      if (g >= 2 && !(ok = wait_all(a_empty + b, ((g >> 1) - 1) & 1))) break;
+      const __half2 ss = __half2half2(s_at(s)[t]);
+      // 1024 + z as fp16: the unpacked words below hold 1024 + q (exponent bits
+      // 0x6400 with q in the low mantissa bits), so one subtraction gives q - z exactly
+      const __half zh = __ushort_as_half(static_cast<unsigned short>(0x6400u | z_at(s)[t]));
+      const __half2 zz = __half2half2(zh);
+      const uint32_t* wrow = w_at(s);
+      uint32_t pk[64];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t word = wrow[i * C::BN + t];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          // bits 4j..4j+3 (weight 8i+2j) into the low half, bits 16+4j.. (8i+2j+1) into the high half
+          const uint32_t v = ((word >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+          const __half2 h = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v), zz), ss);
+          pk[4 * i + j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + s);         // this warp's words, scale and zero are read
+      tmem_st32(tmem_base + lane_off + C::T_A + 64 * b, pk);
+      tmem_st32(tmem_base + lane_off + C::T_A + 64 * b + 32, pk + 32);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(a_full + b);
+    }
+    if (ok) ok = wait_all(done, 0);
+    if (ok) {
+      tc_fence_after();
+      __half* ycol = p.y + n0 + t;
+      for (int c0 = 0; c0 < mpad; c0 += 16) {
+        uint32_t v[16];
+        tmem_ld16(tmem_base + lane_off + C::T_D + c0, v);
+        tmem_ld_wait<16>(v);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int m = c0 + i;
+          if (m < p.M) ycol[static_cast<size_t>(m) * p.N] = __float2half_rn(__uint_as_float(v[i]));
+        }
+      }
+    } else if (lane == 0) {
+      record_timeout();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::TMEM_COLS);
+}
+
+}  // namespace attn

@@ -15,7 +15,7 @@ HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 def declared_symbols():
     text = "".join(open(h).read() for h in HEADERS)
-    return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", text)))
+    return sorted(set(re.findall(r"ATTN_API\s+[\w\s\*]+?\b((?:attn|w4a16)_\w+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module")
@@ -129,3 +129,20 @@ def test_bwd_argument_validation(lib):
     assert call(14, 96) == lib.ATTN_ERR_UNSUPPORTED
     assert call(6, FAKE + 8) == lib.ATTN_ERR_MISALIGNED
     assert call(9, FAKE + 4) == lib.ATTN_ERR_MISALIGNED
+
+
+def test_w4a16_argument_validation(lib):
+    f = lib.w4a16_gemm
+    ok = [FAKE] * 5 + [16, 256, 512, None]
+
+    def call(i=None, val=None):
+        a = list(ok)
+        if i is not None:
+            a[i] = val
+        return f(*a)
+    assert call(1, None) == lib.ATTN_ERR_INVALID_ARG
+    assert call(5, 0) == lib.ATTN_ERR_INVALID_ARG
+    assert call(5, 129) == lib.ATTN_ERR_UNSUPPORTED       # M above 128
+    assert call(6, 200) == lib.ATTN_ERR_UNSUPPORTED       # N not a multiple of 128
+    assert call(7, 100) == lib.ATTN_ERR_UNSUPPORTED       # K not a multiple of 128
+    assert call(4, FAKE + 2) == lib.ATTN_ERR_MISALIGNED

@@ -124,6 +124,42 @@ def make_workload(w: Workload):
     return res
 
 
+@dataclasses.dataclass(frozen=True)
+class GemmWorkload:
+    """A W4A16 GEMM: Y[M, N] = X[M, K] W[K, N] with 4-bit weights."""
+    name: str
+    M: int
+    N: int
+    K: int
+    seed: int = 0
+
+    @property
+    def flops(self) -> float:
+        return 2.0 * self.M * self.N * self.K
+
+
+# decode with a 70B-class model: 16 tokens through one MLP projection
+# (hidden 8192 -> intermediate 28672), the weight-bandwidth-bound case of the
+# pages' quantisation section
+GEMM_WORKLOADS = {
+    "w4a16_decode_mlp": GemmWorkload("w4a16_decode_mlp", 16, 28672, 8192, seed=1006),
+}
+
+
+def make_w4a16(M: int, N: int, K: int, seed: int):
+    """Random W4A16 operands (CPU): x fp16 [M, K] iid N(0, 1); qweight int32
+    [K/8, N] uniform random words (every nibble an independent uniform code
+    0..15); scales fp16 [K/128, N] uniform in [0.005, 0.02); zeros uint8
+    [K/128, N] uniform 0..15."""
+    gen = torch.Generator(device="cpu")
+    gen.manual_seed(seed)
+    x = torch.randn((M, K), generator=gen, dtype=torch.float32).to(torch.float16)
+    qweight = torch.randint(-2**31, 2**31, (K // 8, N), generator=gen, dtype=torch.int64).to(torch.int32)
+    scales = (torch.rand((K // 128, N), generator=gen) * 0.015 + 0.005).to(torch.float16)
+    zeros = torch.randint(0, 16, (K // 128, N), generator=gen, dtype=torch.int64).to(torch.uint8)
+    return x, qweight, scales, zeros
+
+
 def sample_rows(N: int, count: int, seed: int):
     """Sorted distinct query rows to check at full size: the first and last 128
     rows, the rows on either side of every 128-row block boundary that falls in
