@@ -32,6 +32,7 @@ SIGNATURES = {
     "attn_fwd_inject_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, ctypes.c_ulonglong, _P]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "w4a16_gemm": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_abi_version": (_I, []),
@@ -83,6 +84,15 @@ def attn_bwd_workspace_bytes(B, H, N, d):
 
 def w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream):
     return load().w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream)
+
+
+def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, stream):
+    """attn_bwd with its scratch in a fixed array inside the library, for callers
+    that cannot allocate device memory (include/attn_b200.h)."""
+    return load().attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, stream)
+
+
+ATTN_BWD_NOALLOC_MAX_ROWS = 1 << 21
 
 
 def attn_fwd_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit, wait_limit_cycles, stream):

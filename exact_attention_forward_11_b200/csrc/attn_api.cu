@@ -19,6 +19,12 @@
 #include "fp8_prep_kernel.cuh"
 #include "w4a16_kernel.cuh"
 
+// Scratch of attn_bwd_noalloc (D_i, 4 bytes per row) for at most
+// ATTN_BWD_NOALLOC_MAX_ROWS rows: an 8 MiB array that every GPU which loads this
+// library holds until the process exits. In host code its name is only a
+// stand-in: the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) float g_bwd_noalloc_scratch[ATTN_BWD_NOALLOC_MAX_ROWS];
+
 namespace {
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -229,6 +235,23 @@ attn_status launch_bwd(const void* q, const void* k, const void* v, const void* 
 // Bytes of workspace attn_bwd needs: D_i for every row, fp32, rounded to 256.
 size_t bwd_workspace_bytes(long long BH, long long N) { return static_cast<size_t>((BH * N * 4 + 255) / 256 * 256); }
 
+// ---- attn_bwd_noalloc: the backward with its scratch in a fixed device array
+// Device address of g_bwd_noalloc_scratch on the current device. The name is a
+// host-side stand-in in host code, so the address is asked of the runtime once
+// per device (with that device current) and cached; nullptr if that fails.
+float* noalloc_scratch_on_current_device() {
+  static std::atomic<float*> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  float* ptr = cache[dev].load(std::memory_order_acquire);
+  if (ptr != nullptr) return ptr;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_bwd_noalloc_scratch) != cudaSuccess || addr == nullptr) return nullptr;
+  ptr = static_cast<float*>(addr);
+  cache[dev].store(ptr, std::memory_order_release);
+  return ptr;
+}
+
 }  // namespace
 
 extern "C" {
@@ -392,6 +415,29 @@ attn_status w4a16_gemm(const void* x, const void* qweight, const void* scales, c
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                             const void* dout, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                             float scale, int causal, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr || dout == nullptr ||
+      dq == nullptr || dk == nullptr || dv == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = resolve_scale(scale, d); s != ATTN_OK) return s;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(B) * H * N > ATTN_BWD_NOALLOC_MAX_ROWS) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return ATTN_ERR_MISALIGNED;
+  float* dd = noalloc_scratch_on_current_device();
+  if (dd == nullptr) return ATTN_ERR_CUDA;
+  // every row of D that the kernels read is written by the first launch of
+  // this call: nothing in the array has to start at zero
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (d == 128) return launch_bwd<128>(q, k, v, o, lse, dout, dq, dk, dv, dd, B * H, N, scale, causal, st);
+  return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, dd, B * H, N, scale, causal, st);
 }
 
 attn_status attn_get_device_status(void* stream) {

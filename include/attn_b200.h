@@ -158,6 +158,35 @@ ATTN_API attn_status attn_bwd(const void* q, const void* k, const void* v, const
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int H, int N, int d);
 
 /*
+ * attn_bwd_noalloc - attn_bwd for callers that cannot allocate device memory.
+ * (No counterpart in the paper: this is a deployment variant, not part of the
+ * method.) Some callers of this library cannot call cudaMalloc on the path that
+ * runs the backward pass: an operator plugin inside a framework that owns the
+ * whole device memory pool and hands its plugins no scratch buffer, or a
+ * latency-critical service that must not allocate there because cudaMalloc can
+ * synchronise the device and stall every other stream. For them this entry
+ * point takes the same arguments as attn_bwd minus the workspace and keeps its
+ * scratch (D_i, 4 bytes per row) in a fixed array inside the library instead.
+ *   - Limit: B * H * N <= ATTN_BWD_NOALLOC_MAX_ROWS (2^21 rows, an 8 MiB array
+ *     that every GPU which loads the library holds until the process exits);
+ *     larger shapes return ATTN_ERR_UNSUPPORTED without launching anything.
+ *   - The first call on a device looks up the array's device address (once
+ *     per device, with that device current) and caches it; if that lookup
+ *     fails the call returns ATTN_ERR_CUDA. Make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents
+ *     (each call rewrites every row it reads before reading it, so nothing has
+ *     to start at zero). Calls that overlap on the GPU (other streams, other
+ *     threads) race on it: serialise them.
+ *   - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ * Other arguments, results and errors as for attn_bwd.
+ */
+#define ATTN_BWD_NOALLOC_MAX_ROWS (1 << 21)
+ATTN_API attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                             const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                             int B, int H, int N, int d, float scale, int causal, void* stream);
+
+/*
  * attn_get_device_status - synchronises `stream`, then reads and clears the
  * device status word that kernels set when a pipeline wait timed out.
  * Returns ATTN_OK, ATTN_ERR_TIMEOUT, or ATTN_ERR_CUDA if the read failed.
