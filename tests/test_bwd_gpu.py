@@ -17,7 +17,7 @@ import pytest
 import torch
 
 import workloads
-from oracle import attention_bwd_fp64
+from oracle import attention_bwd_fp64, attention_fp64
 
 pytestmark = pytest.mark.gpu
 
@@ -93,14 +93,28 @@ def test_bwd_small_parity(cuda_lib, shape, causal):
 
 
 def test_bwd_custom_scale_and_outliers(cuda_lib):
-    q, k, v = workloads.make_qkv(1, 2, 300, 128, seed=91, outliers=("q", "k"))
-    dout = make_dout(1, 2, 300, 128, seed=5)
+    """Magnitude-20 Q/K outliers make rows so peaked that dP - D cancels: the error
+    of D taken from a bf16 O (2^-9 of sum |dO||O|) then dominates dS. The method
+    takes O as an input, so here both sides get the same O, the oracle's own
+    rounded to bf16 (and its LSE), and the oracle forms D from it as well."""
+    dev = torch.device("cuda:0")
+    B, H, N, d = 1, 2, 300, 128
+    q, k, v = workloads.make_qkv(B, H, N, d, seed=91, outliers=("q", "k"))
+    dout = make_dout(B, H, N, d, seed=5)
     for scale, causal in ((0.03, False), (0.2, True)):
-        dq, dk, dv = run_bwd(cuda_lib, q, k, v, dout, causal, scale=scale)
-        rq, rk, rv = attention_bwd_fp64(f64(q), f64(k), f64(v), f64(dout), scale, causal)
-        check(dq, rq, "dq")
-        check(dk, rk, "dk")
-        check(dv, rv, "dv")
+        o_ref, l_ref = attention_fp64(f64(q), f64(k), f64(v), scale, causal)
+        o_in = torch.from_numpy(o_ref).to(torch.bfloat16)
+        l_in = torch.from_numpy(l_ref).to(torch.float32)
+        g = [Guarded((B, H, N, d), dev) for _ in range(3)]
+        cuda_lib.backward(*(x.to(dev) for x in (q, k, v, o_in)), l_in.to(dev), dout.to(dev), causal=causal,
+                          scale=scale, dq=g[0].t, dk=g[1].t, dv=g[2].t)
+        torch.cuda.synchronize()
+        assert all(x.intact() for x in g)
+        assert cuda_lib.attn_get_device_status(None) == cuda_lib.ATTN_OK
+        rq, rk, rv = attention_bwd_fp64(f64(q), f64(k), f64(v), f64(dout), scale, causal, o=f64(o_in))
+        check(g[0].t.float().cpu().numpy(), rq, "dq")
+        check(g[1].t.float().cpu().numpy(), rk, "dk")
+        check(g[2].t.float().cpu().numpy(), rv, "dv")
 
 
 def test_bwd_closed_forms(cuda_lib):

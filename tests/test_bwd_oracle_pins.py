@@ -129,3 +129,22 @@ def test_row_selection():
     dqs, dks, dvs = attention_bwd_fp64(q, k, v, do, 0.5, True, rows=[0, 7, 39])
     np.testing.assert_array_equal(dqs, dq[:, :, [0, 7, 39]])
     np.testing.assert_array_equal(dks, dk)
+
+
+def test_given_output_enters_through_d_only():
+    """With o = the exact O the result is unchanged; a perturbed o changes only
+    D, so dV is untouched and dQ moves by exactly -scale * dD_i * (P K)_i."""
+    N, d = 9, 4
+    q, k, v, do = (RNG.standard_normal((1, 1, N, d)) for _ in range(4))
+    scale = 0.5
+    o, _ = attention_fp64(q, k, v, scale, False)
+    base = attention_bwd_fp64(q, k, v, do, scale, False)
+    same = attention_bwd_fp64(q, k, v, do, scale, False, o=o)
+    for a, b in zip(base, same):
+        np.testing.assert_allclose(a, b, atol=1e-14)
+    delta = RNG.standard_normal(o.shape) * 1e-3
+    dq2, _, dv2 = attention_bwd_fp64(q, k, v, do, scale, False, o=o + delta)
+    np.testing.assert_allclose(dv2, base[2], atol=1e-15)
+    dd = (do * delta).sum(-1)                                    # change of D_i
+    pk, _ = attention_fp64(q, k, k, scale, False)                # (P K)_i
+    np.testing.assert_allclose(dq2 - base[0], -scale * dd[..., None] * pk, atol=1e-13)
