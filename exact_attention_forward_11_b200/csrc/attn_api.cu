@@ -400,7 +400,7 @@ attn_status w4a16_gemm(const void* x, const void* qweight, const void* scales, c
       !encode_matrix_map(&tz, zeros, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, N, K / C::GROUP, C::BN, 1, false))
     return ATTN_ERR_CUDA;
   const int smem = C::smem_bytes(mpad);
-  if (!set_smem_once(reinterpret_cast<const void*>(attn::w4a16_gemm_sm100), C::smem_bytes(C::MAX_M), 9))
+  if (!set_smem_once(reinterpret_cast<const void*>(attn::w4a16_gemm_sm100), C::max_smem_bytes(), 9))
     return ATTN_ERR_CUDA;
   attn::W4Params p;
   p.M = M;

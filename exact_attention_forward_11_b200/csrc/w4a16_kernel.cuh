@@ -20,7 +20,7 @@
 // from TMEM; only the small X slice is read from shared memory by the MMA.
 //
 // CTA: 8 warps. warp 0 TMA producer (weight words, scales, zero points and the X
-// slice of each K slice into a 4-stage ring), warp 1 MMA issuer (owns TMEM),
+// slice of each K slice into a ring of up to 8 stages), warp 1 MMA issuer (owns TMEM),
 // warps 2-3 idle, warps 4-7 dequantise (thread t: column n0 + t) and write Y.
 // TMEM: two 64-column A buffers (a 128-deep slice of fp16 pairs) and the
 // MPAD-column fp32 accumulator. Every wait is bounded (Waiter).
@@ -37,7 +37,7 @@ namespace attn {
 
 struct W4Cfg {
   static constexpr int THREADS = 256;
-  static constexpr int NST = 4;
+  static constexpr int MAX_NST = 8;            // ring stages: as many as ~110 KB of shared memory holds
   static constexpr int GROUP = 128;            // k per scale / zero point = k per slice
   static constexpr int BN = 128;               // output columns per CTA
   static constexpr int WQ_BYTES = 16 * BN * 4; // 16 words (128 k) x 128 columns
@@ -52,8 +52,22 @@ struct W4Cfg {
   __host__ __device__ static constexpr int stage_bytes(int mpad) {
     return ((2 * x_chunk(mpad) + WQ_BYTES + S_BYTES + Z_BYTES) + 1023) / 1024 * 1024;
   }
-  __host__ __device__ static constexpr int bar_offset(int mpad) { return NST * stage_bytes(mpad); }
-  __host__ __device__ static constexpr int smem_bytes(int mpad) { return bar_offset(mpad) + 16 * 8 + 16 + 1024; }
+  // stages in flight: 8 for small M (two CTAs per SM then keep ~200 KB of weights in
+  // flight per SM), fewer as the X slice grows
+  __host__ __device__ static constexpr int nst(int mpad) {
+    return (110 * 1024) / stage_bytes(mpad) < 2 ? 2
+           : ((110 * 1024) / stage_bytes(mpad) > MAX_NST ? MAX_NST : (110 * 1024) / stage_bytes(mpad));
+  }
+  __host__ __device__ static constexpr int bar_offset(int mpad) { return nst(mpad) * stage_bytes(mpad); }
+  __host__ __device__ static constexpr int smem_bytes(int mpad) {
+    return bar_offset(mpad) + (2 * MAX_NST + 6) * 8 + 16 + 1024;
+  }
+  // the largest smem_bytes over every M (the kernel attribute must cover all)
+  __host__ static constexpr int max_smem_bytes() {
+    int m = 0;
+    for (int mp = 16; mp <= MAX_M; mp += 16) m = smem_bytes(mp) > m ? smem_bytes(mp) : m;
+    return m;
+  }
 };
 
 struct W4Params {
@@ -75,13 +89,14 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
   const int SB = C::stage_bytes(mpad);
   const int XC = C::x_chunk(mpad);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::bar_offset(mpad));
+  const int NST = C::nst(mpad);
   uint64_t* full = bars;                     // NST: TMA bytes
-  uint64_t* empty = full + C::NST;           // NST: MMA commit (X read) + 4 dequant warps (words read)
-  uint64_t* a_full = empty + C::NST;         // 2: 4 dequant warps
+  uint64_t* empty = full + C::MAX_NST;       // NST: MMA commit (X read) + 4 dequant warps (words read)
+  uint64_t* a_full = empty + C::MAX_NST;     // 2: 4 dequant warps
   uint64_t* a_empty = a_full + 2;            // 2: MMA commit
   uint64_t* done = a_empty + 2;              // 1
   uint64_t* drain_bar = done + 1;            // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::MAX_NST + 6);
   uint32_t* abort_word = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -94,7 +109,7 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
   auto z_at = [&](int s) { return smem + s * SB + 2 * XC + C::WQ_BYTES + C::S_BYTES; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::NST; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 5);
     }
@@ -134,8 +149,8 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     const uint32_t bytes = static_cast<uint32_t>(2 * XC + C::WQ_BYTES + C::S_BYTES + C::Z_BYTES);
     int g = 0;
     for (; g < G; ++g) {
-      const int s = g % C::NST;
-      if (g >= C::NST && !(ok = wait_all(empty + s, ((g / C::NST) - 1) & 1))) break;
+      const int s = g % NST;
+      if (g >= NST && !(ok = wait_all(empty + s, ((g / NST) - 1) & 1))) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(full + s, bytes);
         tma_load_3d(x_at(s), &tm_x, full + s, g * C::GROUP, 0, 0, pol_x);
@@ -149,8 +164,8 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     if (!ok) {
       if (lane == 0) record_timeout();
       const uint64_t t0 = sm_clock();
-      for (int j = (g > C::NST ? g - C::NST : 0); j < g; ++j)
-        while (!mbar_try_wait(full + (j % C::NST), (j / C::NST) & 1) && sm_clock() - t0 < p.timeout_cycles) {
+      for (int j = (g > NST ? g - NST : 0); j < g; ++j)
+        while (!mbar_try_wait(full + (j % NST), (j / NST) & 1) && sm_clock() - t0 < p.timeout_cycles) {
         }
     }
   } else if (warp == 1) {
@@ -160,8 +175,8 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     constexpr uint32_t hi = smem_desc_hi(1024);
     const uint32_t x_lo = smem_desc_lo(smem_addr(smem), 16);
     for (int g = 0; g < G; ++g) {
-      const int s = g % C::NST, b = g & 1;
-      if (!(ok = wait_all(full + s, (g / C::NST) & 1))) break;
+      const int s = g % NST, b = g & 1;
+      if (!(ok = wait_all(full + s, (g / NST) & 1))) break;
       if (!(ok = wait_all(a_full + b, (g >> 1) & 1))) break;
       tc_fence_after();
       const uint32_t xa = x_lo + ((s * SB) >> 4);
@@ -187,8 +202,8 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     const int t = wq * 32 + lane;                    // output column n0 + t, TMEM lane t
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     for (int g = 0; g < G; ++g) {
-      const int s = g % C::NST, b = g & 1;
-      if (!(ok = wait_all(full + s, (g / C::NST) & 1))) break;
+      const int s = g % NST, b = g & 1;
+      if (!(ok = wait_all(full + s, (g / NST) & 1))) break;
       if (g >= 2 && !(ok = wait_all(a_empty + b, ((g >> 1) - 1) & 1))) break;
       const __half2 ss = __half2half2(s_at(s)[t]);
       // 1024 + z as fp16: the unpacked words below hold 1024 + q (exponent bits
