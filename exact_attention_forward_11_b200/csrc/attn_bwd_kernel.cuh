@@ -342,8 +342,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (!(ok = wait_all(q_full + s, (it / C::NST) & 1))) break;
       if (!(ok = wait_all(s_full, it & 1))) break;
       tc_fence_after();
-      const float* lse2 = stage_lse(s);
-      const float* dd = stage_dd(s);
+      // the block's statistics are the same for every thread: 16-byte broadcast loads
+      const float4* lse2 = reinterpret_cast<const float4*>(stage_lse(s));
+      const float4* dd = reinterpret_cast<const float4*>(stage_dd(s));
       float pr[128];
       {
         uint32_t sr[128];
@@ -355,9 +356,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         // visible: key < N, and for the diagonal block of a causal launch, key <= query
         const int first_visible = (key >= p.N) ? 128 : ((p.causal && i == jb) ? r : 0);
 #pragma unroll
-        for (int j = 0; j < 128; ++j) {
-          const float x = ex2_approx(fmaf(__uint_as_float(sr[j]), c, -lse2[j]));
-          pr[j] = (j >= first_visible) ? x : 0.f;
+        for (int j4 = 0; j4 < 32; ++j4) {
+          const float4 l4 = lse2[j4];
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * j4 + e;
+            const float x = ex2_approx(fmaf(__uint_as_float(sr[j]), c, -lv[e]));
+            pr[j] = (j >= first_visible) ? x : 0.f;
+          }
         }
         uint32_t pk[64];
 #pragma unroll
@@ -378,10 +385,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tmem_ld_wait<32>(dp);
         uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 16; j += 2) {
           const int q0 = 32 * ch + 2 * j;
-          pk[j] = pack_bf16x2(pr[q0] * (__uint_as_float(dp[2 * j]) - dd[q0]),
-                              pr[q0 + 1] * (__uint_as_float(dp[2 * j + 1]) - dd[q0 + 1]));
+          const float4 d4 = dd[q0 >> 2];
+          pk[j] = pack_bf16x2(pr[q0] * (__uint_as_float(dp[2 * j]) - d4.x),
+                              pr[q0 + 1] * (__uint_as_float(dp[2 * j + 1]) - d4.y));
+          pk[j + 1] = pack_bf16x2(pr[q0 + 2] * (__uint_as_float(dp[2 * j + 2]) - d4.z),
+                                  pr[q0 + 3] * (__uint_as_float(dp[2 * j + 3]) - d4.w));
         }
         tmem_st16(t_dp + 16 * ch, pk);   // dS^T over the dP^T columns already read
       }

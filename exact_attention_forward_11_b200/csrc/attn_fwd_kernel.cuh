@@ -20,8 +20,9 @@
 //   warps 4-7  softmax group for Q tile 1
 //   warp  8    TMA producer (one elected lane)
 //   warp  9    MMA issuer (one elected lane); owns the TMEM allocation
-//   warps 10-11 idle (they complete the control warpgroup, whose registers are
-//              handed to the softmax warpgroups)
+//   warps 10-11 FP8 (f16 P V): convert each E4M3 V tile to f16 in shared memory;
+//              otherwise idle (they complete the control warpgroup, whose
+//              registers are handed to the softmax warpgroups)
 // TMEM (512 columns x 128 lanes of 32 bit):
 //   S_t  columns [128 t, 128 t + 128)   fp32 scores of tile t; P_t (bf16 pairs or
 //                                        E4M3 quads) is written over its first
@@ -62,15 +63,27 @@ struct FwdCfg {
   static constexpr int CHUNKS = D / SW_COLS;                    // 128-byte column chunks per row
   static constexpr int CHUNK_BYTES = 128 * 128;                 // one chunk of a 128-row tile
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;       // one 128-row tile of Q, K or V
-  static constexpr int NSLOT = (TILE_BYTES == 32768) ? 4 : 8;   // K/V ring slots
-  static constexpr int UMMA_K = FP8 ? 32 : 16;                  // K elements per MMA
+  // FP8 P V in 16-bit: the two idle control warps convert each E4M3 V tile to an
+  // f16 tile in shared memory (exact: every E4M3 value is an f16 value) and P is
+  // written as f16 pairs, so P V is a kind::f16 MMA with one term (the
+  // alternative keeps V in E4M3 and writes P as two E4M3 terms hi + lo, K = 256)
+#ifndef ATTN_FP8_PV_F16
+#define ATTN_FP8_PV_F16 1
+#endif
+  static constexpr bool PV_F16 = FP8 && (ATTN_FP8_PV_F16 != 0);
+  static constexpr bool PV_HILO = FP8 && !PV_F16;
+  static constexpr int NSLOT = (TILE_BYTES == 32768) ? 4 : (PV_F16 ? 6 : 8);   // K/V ring slots
+  static constexpr int UMMA_K = FP8 ? 32 : 16;                  // K elements per S MMA
   static constexpr int S_KSTEPS = D / UMMA_K;
-  static constexpr int PV_KSTEPS = kBlockN / UMMA_K;
-  // P in TMEM: bf16 pairs (64 columns), or for FP8 two E4M3 terms hi + lo of
-  // each value (32 + 32 columns), so the P V product sees ~7 significant bits
-  // of P instead of E4M3's 4; P V then runs over K = 256 (hi | lo) x (V ; V).
+  static constexpr int PV_UMMA_K = PV_HILO ? 32 : 16;           // K elements (keys) per P V MMA
+  static constexpr int PV_KSTEPS = kBlockN / PV_UMMA_K;
+  // P in TMEM: 16-bit pairs (64 columns), or for the hi/lo form two E4M3 terms
+  // of each value (32 + 32 columns), so the P V product sees ~7 significant
+  // bits of P instead of E4M3's 4; P V then runs over K = 256 (hi | lo) x (V ; V).
   static constexpr int P_COLS = 64;
-  static constexpr int PV_KSTEPS_TOTAL = FP8 ? 2 * PV_KSTEPS : PV_KSTEPS;
+  static constexpr int PV_KSTEPS_TOTAL = PV_HILO ? 2 * PV_KSTEPS : PV_KSTEPS;
+  static constexpr int VCONV_BYTES = PV_F16 ? 2 * 128 * 128 : 0;   // one f16 V tile (2 chunks)
+  static constexpr int VCONV_BUFS = PV_F16 ? 2 : 0;
   // P is handed to the MMA in P_CHUNKS chunks of 64 keys, each with its own
   // barrier, so P V of a tile starts under the tile's remaining exponentials.
 #ifndef ATTN_P_CHUNKS
@@ -96,8 +109,8 @@ struct FwdCfg {
 #ifndef ATTN_FP8_RESCALE_THRESHOLD
 #define ATTN_FP8_RESCALE_THRESHOLD 0.8f
 #endif
-  static constexpr float RESCALE_THRESHOLD = FP8 ? ATTN_FP8_RESCALE_THRESHOLD : 8.0f;
-  static constexpr float P_PRESCALE_LOG2 = 8.0f;  // FP8 only
+  static constexpr float RESCALE_THRESHOLD = PV_HILO ? ATTN_FP8_RESCALE_THRESHOLD : 8.0f;
+  static constexpr float P_PRESCALE_LOG2 = PV_HILO ? 8.0f : 0.0f;  // E4M3 P only
   // Pairs of P values (by index mod 8) whose exp2 runs as a polynomial on the
   // FMA pipe instead of the MUFU unit, in blocks that need no masking. MUFU
   // throughput alone (16/clk/SM) matches the tensor cores at d = 128, so part
@@ -113,8 +126,9 @@ struct FwdCfg {
   // shared memory map (offsets from a 1024-aligned base)
   static constexpr int SMEM_Q = 0;
   static constexpr int SMEM_KV = SMEM_Q + Q_TILES * TILE_BYTES;
-  static constexpr int SMEM_BAR = SMEM_KV + NSLOT * TILE_BYTES;
-  static constexpr int NUM_BARS = 2 + 2 * NSLOT + (2 + P_CHUNKS) * Q_TILES + 1;
+  static constexpr int SMEM_VCONV = SMEM_KV + NSLOT * TILE_BYTES;
+  static constexpr int SMEM_BAR = SMEM_VCONV + VCONV_BUFS * VCONV_BYTES;
+  static constexpr int NUM_BARS = 2 + 2 * NSLOT + (2 + P_CHUNKS) * Q_TILES + 1 + 2 * VCONV_BUFS;
   static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;  // + alignment slack
 };
@@ -208,7 +222,7 @@ __device__ __forceinline__ float row_max128(const uint32_t (&sr)[128]) { return 
 // pk; adds the fp32 values to the packed accumulators. The scale-and-subtract
 // is a scalar FMA per element (a packed FMA would compete with MUFU for issue);
 // the sums use packed adds, which do not.
-template <uint32_t POLY_MASK, int PAIRS = 16>
+template <uint32_t POLY_MASK, int PAIRS = 16, bool F16 = false>
 __device__ __forceinline__ void p_chunk_bf16(const uint32_t* sr, int ch, float c, float m,
                                              uint64_t (&acc)[4], uint32_t (&pk)[PAIRS]) {
   using namespace b200;
@@ -218,7 +232,7 @@ __device__ __forceinline__ void p_chunk_bf16(const uint32_t* sr, int ch, float c
     float p0, p1;
     exp2_pair<POLY_MASK>(fmaf(__uint_as_float(sr[k]), c, -m), fmaf(__uint_as_float(sr[k + 1]), c, -m), i, p0, p1);
     acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-    pk[i] = pack_bf16x2(p0, p1);
+    pk[i] = F16 ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
   }
 }
 
@@ -271,9 +285,9 @@ __device__ __forceinline__ float p_row_to_tmem(const uint32_t (&sr)[128], float 
   constexpr int COLS = 64 / C::P_CHUNKS;   // TMEM columns of P per chunk (bf16 pairs / hi+lo quads)
 #pragma unroll
   for (int ch = 0; ch < C::P_CHUNKS; ++ch) {
-    if constexpr (!C::FP8) {
+    if constexpr (!C::PV_HILO) {
       uint32_t pk[COLS];
-      p_chunk_bf16<POLY_MASK, COLS>(sr, ch, c, m, acc, pk);
+      p_chunk_bf16<POLY_MASK, COLS, C::PV_F16>(sr, ch, c, m, acc, pk);
       if (ch > 0) {
         release_chunk(p_full_t + ch - 1);
       }
@@ -359,6 +373,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* o_done = p_full + C::Q_TILES * C::P_CHUNKS;  // Q_TILES
   uint64_t* drain_bar = o_done + C::Q_TILES;     // 1
   uint64_t* q_empty = drain_bar + 1;             // 1
+  uint64_t* vconv_full = q_empty + 1;            // VCONV_BUFS (f16 V tile written: 2 converter warps)
+  uint64_t* vconv_empty = vconv_full + C::VCONV_BUFS;  // VCONV_BUFS (its P V MMAs done: MMA commit)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
   uint32_t* abort_word = tmem_slot + 1;
 
@@ -372,7 +388,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(q_empty, 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(kv_full + i, 1);
-      mbar_init(kv_empty + i, 1);
+      // slots alternate K, V (NSLOT is even); with the f16 V conversion the two
+      // converter warps, not the MMA, are the last readers of a V slot
+      mbar_init(kv_empty + i, (C::PV_F16 && (i & 1)) ? 2 : 1);
+    }
+    for (int b = 0; b < C::VCONV_BUFS; ++b) {
+      mbar_init(vconv_full + b, 2);
+      mbar_init(vconv_empty + b, 1);
     }
     for (int t = 0; t < C::Q_TILES; ++t) {
       mbar_init(s_full + t, 1);
@@ -474,16 +496,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     };
     const uint32_t leader = elect_one() ? 1u : 0u;
     auto commit = [&](uint64_t* bar) { mma_commit(bar, leader); };
-    constexpr uint32_t fmt = C::FP8 ? 0u : 1u;
+    constexpr uint32_t fmt = C::FP8 ? 0u : 1u;                 // e4m3 (kind::f8f6f4) / bf16
+    constexpr uint32_t fmt_o = C::PV_F16 ? 0u : fmt;           // f16 P V: kind::f16 with f16 operands
     constexpr uint32_t idesc_s = instr_desc(fmt, 128, kBlockN, 0, 0);
-    constexpr uint32_t idesc_o = instr_desc(fmt, 128, C::D, 0, 1);
+    constexpr uint32_t idesc_o = instr_desc(fmt_o, 128, C::D, 0, 1);
     // Descriptor words, computed once: per k-step and per slot only the low
     // word moves (by a compile-time or per-slot constant).
     constexpr uint32_t hi_kmaj = smem_desc_hi(1024);   // 8 rows x 128 B per swizzle atom
     constexpr uint32_t hi_mnmaj = smem_desc_hi(1024);
     const uint32_t q_lo = smem_desc_lo(smem_addr(smem + C::SMEM_Q), 16);
     const uint32_t k_lo = smem_desc_lo(smem_addr(smem + C::SMEM_KV), 16);
-    const uint32_t v_lo = smem_desc_lo(smem_addr(smem + C::SMEM_KV), C::CHUNK_BYTES);
+    const uint32_t v_lo = C::PV_F16 ? smem_desc_lo(smem_addr(smem + C::SMEM_VCONV), 128 * 128)
+                                    : smem_desc_lo(smem_addr(smem + C::SMEM_KV), C::CHUNK_BYTES);
     // S_t = Q_t K_j^T over D in UMMA_K steps (K-major operands, 128B swizzle)
     auto issue_s = [&](int t, uint32_t slot) {
       const uint32_t qa = q_lo + ((t * C::TILE_BYTES) >> 4);
@@ -502,28 +526,30 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     };
     // O_t (+)= P_t V_j for the keys of P chunk c: P from TMEM (over S_t), V
-    // MN-major in shared memory. bf16: K=16 steps; FP8: the hi and the lo steps
-    // of the chunk's keys.
+    // MN-major in shared memory. bf16 and f16 P: K=16 steps over the V slot (or
+    // the converted f16 V buffer `slot`); E4M3 P: the hi and the lo steps of the
+    // chunk's keys.
     auto issue_pv_chunk = [&](int t, uint32_t slot, int c, bool acc) {
-      const uint32_t va = v_lo + ((slot * C::TILE_BYTES) >> 4);
+      const uint32_t va = v_lo + ((slot * (C::PV_F16 ? C::VCONV_BYTES : C::TILE_BYTES)) >> 4);
       const uint32_t o_tmem = tmem_base + C::O_COL0 + t * C::D;
       const uint32_t p_tmem = tmem_base + t * 128;
       constexpr int STEPS = C::PV_KSTEPS / C::P_CHUNKS;   // K steps per chunk per term
 #pragma unroll
-      for (int term = 0; term < (C::FP8 ? 2 : 1); ++term)
+      for (int term = 0; term < (C::PV_HILO ? 2 : 1); ++term)
 #pragma unroll
         for (int i = 0; i < STEPS; ++i) {
           const int kv = c * STEPS + i;                     // K step within V
           const int kk = term * C::PV_KSTEPS + kv;          // K step within [hi | lo]
-          const uint64_t db = smem_desc(va + ((kv * C::UMMA_K * 128) >> 4), hi_mnmaj);
+          const uint64_t db = smem_desc(va + ((kv * C::PV_UMMA_K * 128) >> 4), hi_mnmaj);
           const uint32_t accum = (acc || term > 0 || i > 0) ? 1u : 0u;
-          if constexpr (C::FP8)
+          if constexpr (C::PV_HILO)
             mma_f8_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum, leader);
           else
             mma_f16_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum, leader);
         }
     };
     uint32_t g = 0;                       // K/V tiles consumed so far (same count as the producer's)
+    uint32_t vb = 0;                      // f16 V buffers consumed so far (vconv phases)
     uint32_t pc[C::Q_TILES];              // blocks of P consumed per tile (p_full phases)
 #pragma unroll
     for (int t = 0; t < C::Q_TILES; ++t) pc[t] = 0;
@@ -554,14 +580,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         for (int t = 0; t < C::Q_TILES; ++t) {
           if (j >= w.nkv[t]) continue;
           if (!v_ready) {
-            if (!(ok = wait_all(kv_full + vslot, (vg / C::NSLOT) & 1))) break;
+            if constexpr (C::PV_F16)
+              ok = wait_all(vconv_full + (vb & 1), (vb >> 1) & 1);
+            else
+              ok = wait_all(kv_full + vslot, (vg / C::NSLOT) & 1);
+            if (!ok) break;
             v_ready = true;
           }
 #pragma unroll
           for (int c = 0; c < C::P_CHUNKS; ++c) {
             if (!(ok = wait_all(p_full + t * C::P_CHUNKS + c, pc[t] & 1))) break;
             tc_fence_after();
-            issue_pv_chunk(t, vslot, c, j > 0 || c > 0);
+            issue_pv_chunk(t, C::PV_F16 ? (vb & 1) : vslot, c, j > 0 || c > 0);
           }
           if (!ok) break;
           ++pc[t];
@@ -579,7 +609,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
         }
         if (!ok) break;
-        commit(kv_empty + vslot);
+        if constexpr (C::PV_F16) {
+          commit(vconv_empty + (vb & 1));   // the converted tile's P V MMAs are issued
+          ++vb;
+        } else {
+          commit(kv_empty + vslot);
+        }
         if (any_s) commit(kv_empty + kslot);
         if (any_s && j + 2 == w.nkv_max) commit(q_empty);   // the unit's last S MMAs are issued
       }
@@ -592,7 +627,58 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     drain_wait(drain_bar, 0, p.timeout_cycles);
     __syncwarp();
   } else if (warp > C::MMA_WARP) {
-    regs_decrease<C::REGS_CONTROL>();  // idle warps of the control warpgroup
+    regs_decrease<C::REGS_CONTROL>();
+    if constexpr (C::PV_F16) {
+      // ======================= E4M3 -> f16 V conversion =======================
+      // The two remaining control warps turn each E4M3 V tile (128 keys x 128
+      // bytes, 128-byte swizzle) into an f16 tile of two 64-column chunks with
+      // the same swizzle, the MN-major B operand of the f16 P V MMA. Every E4M3
+      // value is exactly an f16 value. Thread ct handles (row, 16-byte unit)
+      // pairs ct, ct + 64, ...: eight threads read one 128-byte row.
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, waiter.wait(bar, parity));
+      };
+      const int ct = (warp - C::MMA_WARP - 1) * 32 + lane;
+      uint32_t g = 0, vb = 0;
+      bool ok = true;
+      for (int k = 0; ok && k * static_cast<int>(gridDim.x) < p.num_units; ++k) {
+        const int u = unit_of_round(k);
+        if (u >= p.num_units) continue;
+        const UnitInfo<C> w(p, u, QB, NPAIR);
+        for (int j = 0; j < w.nkv_max; ++j, ++vb) {
+          const uint32_t vg = g + 2 * j + 1, vslot = vg % C::NSLOT, b = vb & 1;
+          if (!(ok = wait_all(kv_full + vslot, (vg / C::NSLOT) & 1))) break;
+          if (vb >= 2 && !(ok = wait_all(vconv_empty + b, ((vb >> 1) - 1) & 1))) break;
+          const uint8_t* src = smem + C::SMEM_KV + vslot * C::TILE_BYTES;
+          uint8_t* dst = smem + C::SMEM_VCONV + b * C::VCONV_BYTES;
+#pragma unroll 2
+          for (int i = 0; i < 16; ++i) {
+            const int pr = ct + 64 * i, r = pr >> 3, un = pr & 7;        // key row, 16-code unit (d = 16 un ..)
+            const uint4 c16 = *reinterpret_cast<const uint4*>(src + r * 128 + ((un ^ (r & 7)) << 4));
+            const uint32_t wds[4] = {c16.x, c16.y, c16.z, c16.w};
+            uint32_t h[8];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              h[2 * q] = f16x2_from_e4m3x2(static_cast<uint16_t>(wds[q] & 0xFFFFu));
+              h[2 * q + 1] = f16x2_from_e4m3x2(static_cast<uint16_t>(wds[q] >> 16));
+            }
+            // f16 d = 16 un + e sits in chunk un / 4, 16-byte unit 2 (un % 4) + (e / 8)
+            uint8_t* drow = dst + (un >> 2) * (128 * 128) + r * 128;
+            const int u0 = 2 * (un & 3);
+            *reinterpret_cast<uint4*>(drow + ((u0 ^ (r & 7)) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(drow + (((u0 + 1) ^ (r & 7)) << 4)) = make_uint4(h[4], h[5], h[6], h[7]);
+          }
+          fence_proxy_async_shared();   // the MMA (async proxy) reads what these threads wrote
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(vconv_full + b);
+            mbar_arrive(kv_empty + vslot);   // the E4M3 V slot is read
+          }
+        }
+        g += 2 * w.nkv_max;
+      }
+      if (!ok && lane == 0) record_timeout();
+    }
   } else {
     // ======================= softmax groups =======================
     regs_increase<C::REGS_SOFTMAX>();
@@ -697,7 +783,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       ++oc;
       tc_fence_after();
       float inv_l = 1.f / l_run;
-      if constexpr (C::FP8) inv_l *= v_max * 0.00390625f;  // undo the V ratio and 2^8 pre-scale
+      // undo the V ratio (and the 2^8 pre-scale of E4M3 P)
+      if constexpr (C::FP8) inv_l *= v_max * (C::PV_HILO ? 0.00390625f : 1.0f);
       const bool in_range = row < p.N;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (in_range ? row : 0)) * C::D;
 #pragma unroll
