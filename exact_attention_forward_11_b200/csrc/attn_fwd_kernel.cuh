@@ -24,8 +24,8 @@
 //              otherwise idle (they complete the control warpgroup, whose
 //              registers are handed to the softmax warpgroups)
 // TMEM (512 columns x 128 lanes of 32 bit):
-//   S_t  columns [128 t, 128 t + 128)   fp32 scores of tile t; P_t (bf16 pairs or
-//                                        E4M3 quads) is written over its first
+//   S_t  columns [128 t, 128 t + 128)   fp32 scores of tile t; P_t (bf16 pairs, or
+//                                        f16 pairs for FP8) is written over its first
 //                                        columns once S_t has been read
 //   O_t  columns [256 + D t, 256 + D t + D)   fp32 output accumulator of tile t
 // Shared memory: the Q tiles of the current work unit (reloaded for the next unit
@@ -63,25 +63,19 @@ struct FwdCfg {
   static constexpr int CHUNKS = D / SW_COLS;                    // 128-byte column chunks per row
   static constexpr int CHUNK_BYTES = 128 * 128;                 // one chunk of a 128-row tile
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;       // one 128-row tile of Q, K or V
-  // FP8 P V in 16-bit: the two idle control warps convert each E4M3 V tile to an
-  // f16 tile in shared memory (exact: every E4M3 value is an f16 value) and P is
-  // written as f16 pairs, so P V is a kind::f16 MMA with one term (the
-  // alternative keeps V in E4M3 and writes P as two E4M3 terms hi + lo, K = 256)
-#ifndef ATTN_FP8_PV_F16
-#define ATTN_FP8_PV_F16 1
-#endif
-  static constexpr bool PV_F16 = FP8 && (ATTN_FP8_PV_F16 != 0);
-  static constexpr bool PV_HILO = FP8 && !PV_F16;
+  // FP8 P V in 16 bits: the two otherwise idle control warps convert each E4M3 V
+  // tile to an f16 tile in shared memory (exact: every E4M3 value is an f16
+  // value) and P is written as f16 pairs, so P V is one kind::f16 MMA over the
+  // block's keys. (Measured against P as two E4M3 terms hi + lo over K = 256 with
+  // V kept in E4M3: 15 % faster at the same accuracy.)
+  static constexpr bool PV_F16 = FP8;
   static constexpr int NSLOT = (TILE_BYTES == 32768) ? 4 : (PV_F16 ? 6 : 8);   // K/V ring slots
   static constexpr int UMMA_K = FP8 ? 32 : 16;                  // K elements per S MMA
   static constexpr int S_KSTEPS = D / UMMA_K;
-  static constexpr int PV_UMMA_K = PV_HILO ? 32 : 16;           // K elements (keys) per P V MMA
+  static constexpr int PV_UMMA_K = 16;                          // K elements (keys) per P V MMA
   static constexpr int PV_KSTEPS = kBlockN / PV_UMMA_K;
-  // P in TMEM: 16-bit pairs (64 columns), or for the hi/lo form two E4M3 terms
-  // of each value (32 + 32 columns), so the P V product sees ~7 significant
-  // bits of P instead of E4M3's 4; P V then runs over K = 256 (hi | lo) x (V ; V).
+  // P in TMEM: 16-bit pairs (bf16, or f16 for FP8) over the first 64 columns of S
   static constexpr int P_COLS = 64;
-  static constexpr int PV_KSTEPS_TOTAL = PV_HILO ? 2 * PV_KSTEPS : PV_KSTEPS;
   static constexpr int VCONV_BYTES = PV_F16 ? 2 * 128 * 128 : 0;   // one f16 V tile (2 chunks)
   static constexpr int VCONV_BUFS = PV_F16 ? 2 : 0;
   // P is handed to the MMA in P_CHUNKS chunks of 64 keys, each with its own
@@ -103,14 +97,9 @@ struct FwdCfg {
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t O_COL0 = 256;
   // Lazy rescaling: the running maximum is only moved when a new block raises it
-  // by more than this (log2 units). Exact for any value; 8 keeps bf16 P <= 256.
-  // FP8 P must stay at or below 448 (the largest E4M3 value) after a 2^8
-  // pre-scale: a lag of at most 0.8 keeps it <= 2^8.8 = 445.7.
-#ifndef ATTN_FP8_RESCALE_THRESHOLD
-#define ATTN_FP8_RESCALE_THRESHOLD 0.8f
-#endif
-  static constexpr float RESCALE_THRESHOLD = PV_HILO ? ATTN_FP8_RESCALE_THRESHOLD : 8.0f;
-  static constexpr float P_PRESCALE_LOG2 = PV_HILO ? 8.0f : 0.0f;  // E4M3 P only
+  // by more than this (log2 units). Exact for any value; 8 keeps P <= 256, which
+  // bf16 and f16 both hold.
+  static constexpr float RESCALE_THRESHOLD = 8.0f;
   // Pairs of P values (by index mod 8) whose exp2 runs as a polynomial on the
   // FMA pipe instead of the MUFU unit, in blocks that need no masking. MUFU
   // throughput alone (16/clk/SM) matches the tensor cores at d = 128, so part
@@ -119,7 +108,7 @@ struct FwdCfg {
 #define ATTN_POLY_MASK_BF16 0x00u
 #endif
 #ifndef ATTN_POLY_MASK_FP8
-#define ATTN_POLY_MASK_FP8 0x22u
+#define ATTN_POLY_MASK_FP8 0x00u
 #endif
   static constexpr uint32_t POLY_MASK = FP8 ? ATTN_POLY_MASK_FP8 : ATTN_POLY_MASK_BF16;
 
@@ -165,7 +154,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint6
 // relative error (Remez exchange, fit_exp2_poly.py: max relative error 7.5e-5);
 // 2^n is applied by adding n to the exponent field. Arguments are clamped at
 // -125 so the result stays normal; 2^-125 stands in for 0, far below any P value
-// that survives bf16 / E4M3 rounding next to the row maximum (P <= 2^8).
+// that survives bf16 / f16 rounding next to the row maximum (P <= 2^8).
 constexpr float kExp2C0 = 0.9999280571937561f;
 constexpr float kExp2C1 = 0.6932609677314758f;
 constexpr float kExp2C2 = 0.2426111251115799f;
@@ -236,34 +225,6 @@ __device__ __forceinline__ void p_chunk_bf16(const uint32_t* sr, int ch, float c
   }
 }
 
-// FP8 variant: P = hi + lo, both E4M3: hi = e4m3(p) converted straight from
-// fp32, lo = e4m3(p - hi) with the residual formed in f16x2 (p rounded to f16,
-// hi decoded exactly to f16). The chunk's keys give QUADS hi words and QUADS lo
-// words (four codes each). Conversion forms were chosen by measured contention
-// with MUFU ex2 on B200: e4m3x2 <- f32 +0.2 cycles, f16x2 <- e4m3x2 +0.4,
-// sub.f16x2 +1.2, e4m3x2 <- f16x2 +2.2, f16x2 <- f32 none.
-template <uint32_t POLY_MASK, int QUADS = 8>
-__device__ __forceinline__ void p_chunk_fp8(const uint32_t* sr, int ch, float c, float m,
-                                            uint64_t (&acc)[4], uint32_t (&hi)[QUADS], uint32_t (&lo)[QUADS]) {
-  using namespace b200;
-#pragma unroll
-  for (int i = 0; i < QUADS; ++i) {
-    const int k = 4 * QUADS * ch + 4 * i;
-    float p0, p1, p2, p3;
-    exp2_pair<POLY_MASK>(fmaf(__uint_as_float(sr[k]), c, -m), fmaf(__uint_as_float(sr[k + 1]), c, -m), 2 * i, p0,
-                         p1);
-    exp2_pair<POLY_MASK>(fmaf(__uint_as_float(sr[k + 2]), c, -m), fmaf(__uint_as_float(sr[k + 3]), c, -m), 2 * i + 1,
-                         p2, p3);
-    acc[(2 * i) & 3] = f2_add(acc[(2 * i) & 3], f2_pack(p0, p1));
-    acc[(2 * i + 1) & 3] = f2_add(acc[(2 * i + 1) & 3], f2_pack(p2, p3));
-    const uint16_t hi01 = e4m3x2_from_f32(p0, p1), hi23 = e4m3x2_from_f32(p2, p3);
-    const uint32_t r01 = hsub2_u32(pack_f16x2(p0, p1), f16x2_from_e4m3x2(hi01));
-    const uint32_t r23 = hsub2_u32(pack_f16x2(p2, p3), f16x2_from_e4m3x2(hi23));
-    hi[i] = static_cast<uint32_t>(hi01) | (static_cast<uint32_t>(hi23) << 16);
-    lo[i] = static_cast<uint32_t>(e4m3x2_from_f16x2(r01)) | (static_cast<uint32_t>(e4m3x2_from_f16x2(r23)) << 16);
-  }
-}
-
 // Hands a P chunk to the MMA thread: each thread waits for its own TMEM stores
 // and arrives (the barrier counts the 128 threads of the group).
 __device__ __forceinline__ void release_chunk(uint64_t* bar) {
@@ -285,32 +246,14 @@ __device__ __forceinline__ float p_row_to_tmem(const uint32_t (&sr)[128], float 
   constexpr int COLS = 64 / C::P_CHUNKS;   // TMEM columns of P per chunk (bf16 pairs / hi+lo quads)
 #pragma unroll
   for (int ch = 0; ch < C::P_CHUNKS; ++ch) {
-    if constexpr (!C::PV_HILO) {
-      uint32_t pk[COLS];
-      p_chunk_bf16<POLY_MASK, COLS, C::PV_F16>(sr, ch, c, m, acc, pk);
-      if (ch > 0) {
-        release_chunk(p_full_t + ch - 1);
-      }
-      if constexpr (COLS == 16) tmem_st16(s_tm + COLS * ch, pk);
-      else if constexpr (COLS == 32) tmem_st32(s_tm + COLS * ch, pk);
-      else { tmem_st32(s_tm, pk); tmem_st32(s_tm + 32, pk + 32); }
-    } else {
-      uint32_t hi[COLS / 2], lo[COLS / 2];
-      p_chunk_fp8<POLY_MASK, COLS / 2>(sr, ch, c, m, acc, hi, lo);
-      if (ch > 0) {
-        release_chunk(p_full_t + ch - 1);
-      }
-      if constexpr (COLS == 16) {
-        tmem_st8(s_tm + 8 * ch, hi);
-        tmem_st8(s_tm + 32 + 8 * ch, lo);
-      } else if constexpr (COLS == 32) {
-        tmem_st16(s_tm + 16 * ch, hi);
-        tmem_st16(s_tm + 32 + 16 * ch, lo);
-      } else {
-        tmem_st32(s_tm, hi);
-        tmem_st32(s_tm + 32, lo);
-      }
+    uint32_t pk[COLS];
+    p_chunk_bf16<POLY_MASK, COLS, C::PV_F16>(sr, ch, c, m, acc, pk);
+    if (ch > 0) {
+      release_chunk(p_full_t + ch - 1);
     }
+    if constexpr (COLS == 16) tmem_st16(s_tm + COLS * ch, pk);
+    else if constexpr (COLS == 32) tmem_st32(s_tm + COLS * ch, pk);
+    else { tmem_st32(s_tm, pk); tmem_st32(s_tm + 32, pk + 32); }
   }
   release_chunk(p_full_t + C::P_CHUNKS - 1);
   float a, b;
@@ -526,27 +469,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     };
     // O_t (+)= P_t V_j for the keys of P chunk c: P from TMEM (over S_t), V
-    // MN-major in shared memory. bf16 and f16 P: K=16 steps over the V slot (or
-    // the converted f16 V buffer `slot`); E4M3 P: the hi and the lo steps of the
-    // chunk's keys.
+    // MN-major in shared memory, K = 16 keys per step: the bf16 V slot, or for
+    // FP8 the converted f16 V buffer `slot`.
     auto issue_pv_chunk = [&](int t, uint32_t slot, int c, bool acc) {
       const uint32_t va = v_lo + ((slot * (C::PV_F16 ? C::VCONV_BYTES : C::TILE_BYTES)) >> 4);
       const uint32_t o_tmem = tmem_base + C::O_COL0 + t * C::D;
       const uint32_t p_tmem = tmem_base + t * 128;
       constexpr int STEPS = C::PV_KSTEPS / C::P_CHUNKS;   // K steps per chunk per term
 #pragma unroll
-      for (int term = 0; term < (C::PV_HILO ? 2 : 1); ++term)
-#pragma unroll
-        for (int i = 0; i < STEPS; ++i) {
-          const int kv = c * STEPS + i;                     // K step within V
-          const int kk = term * C::PV_KSTEPS + kv;          // K step within [hi | lo]
-          const uint64_t db = smem_desc(va + ((kv * C::PV_UMMA_K * 128) >> 4), hi_mnmaj);
-          const uint32_t accum = (acc || term > 0 || i > 0) ? 1u : 0u;
-          if constexpr (C::PV_HILO)
-            mma_f8_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum, leader);
-          else
-            mma_f16_ts(o_tmem, p_tmem + kk * 8, db, idesc_o, accum, leader);
-        }
+      for (int i = 0; i < STEPS; ++i) {
+        const int kv = c * STEPS + i;                       // K step within V
+        const uint64_t db = smem_desc(va + ((kv * C::PV_UMMA_K * 128) >> 4), hi_mnmaj);
+        mma_f16_ts(o_tmem, p_tmem + kv * 8, db, idesc_o, (acc || i > 0) ? 1u : 0u, leader);
+      }
     };
     uint32_t g = 0;                       // K/V tiles consumed so far (same count as the producer's)
     uint32_t vb = 0;                      // f16 V buffers consumed so far (vconv phases)
@@ -746,8 +681,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const float m_blk = row_max128(sr) * c;
         float m_use = m_run;
         if (m_blk - m_run > C::RESCALE_THRESHOLD) m_use = m_blk;
-        // exponent offset: FP8 folds the V tile scale ratio and a 2^8 pre-scale in
-        const float m_exp = C::FP8 ? (m_use - v_log2_ratio - C::P_PRESCALE_LOG2) : m_use;
+        // exponent offset: FP8 folds the V tile scale ratio in
+        const float m_exp = C::FP8 ? (m_use - v_log2_ratio) : m_use;
         const bool moved = m_use != m_run;
         // 2^(m_run - m_use); 0 on the first block
         const float alpha = moved ? ex2_approx(m_run - m_use) : 1.f;
@@ -770,7 +705,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         uint64_t* pf = p_full + t * C::P_CHUNKS;
         float sum = masked ? p_row_to_tmem<C, 0u>(sr, c, m_exp, s_tm, pf)
                            : p_row_to_tmem<C, C::POLY_MASK>(sr, c, m_exp, s_tm, pf);
-        if constexpr (C::FP8) sum *= ex2_approx(-v_log2_ratio - C::P_PRESCALE_LOG2);  // units of 2^m_use
+        if constexpr (C::FP8) sum *= ex2_approx(-v_log2_ratio);  // units of 2^m_use
         l_run = l_run * alpha + sum;
         m_run = m_use;
       }
@@ -783,8 +718,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       ++oc;
       tc_fence_after();
       float inv_l = 1.f / l_run;
-      // undo the V ratio (and the 2^8 pre-scale of E4M3 P)
-      if constexpr (C::FP8) inv_l *= v_max * (C::PV_HILO ? 0.00390625f : 1.0f);
+      if constexpr (C::FP8) inv_l *= v_max;   // undo the V ratio folded into P
       const bool in_range = row < p.N;
       __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (in_range ? row : 0)) * C::D;
 #pragma unroll

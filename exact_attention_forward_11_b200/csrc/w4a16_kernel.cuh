@@ -22,8 +22,8 @@
 // CTA: 8 warps. warp 0 TMA producer (weight words, scales, zero points and the X
 // slice of each K slice into a ring of up to 8 stages), warp 1 MMA issuer (owns TMEM),
 // warps 2-3 idle, warps 4-7 dequantise (thread t: column n0 + t) and write Y.
-// TMEM: two 64-column A buffers (a 128-deep slice of fp16 pairs) and the
-// MPAD-column fp32 accumulator. Every wait is bounded (Waiter).
+// TMEM: three (two for M > 64) 64-column A buffers (a 128-deep slice of fp16
+// pairs each) and the MPAD-column fp32 accumulator. Every wait is bounded (Waiter).
 #pragma once
 
 #include <cstdint>
@@ -45,8 +45,12 @@ struct W4Cfg {
   static constexpr int Z_BYTES = BN;
   static constexpr int MAX_M = 128;
   static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t T_A = 0;           // A buffers: [0, 64), [64, 128)
-  static constexpr uint32_t T_D = 128;         // accumulator: MPAD columns
+  static constexpr uint32_t T_A = 0;           // A buffers: 64 columns each from column 0
+  static constexpr int MAX_NA = 3;
+  // A buffers in flight: three when the accumulator (MPAD columns after them)
+  // leaves room in the 256 columns, else two
+  __host__ __device__ static constexpr int na(int mpad) { return mpad <= 64 ? 3 : 2; }
+  __host__ __device__ static constexpr uint32_t t_d(int mpad) { return 64u * na(mpad); }
   // stage layout (offsets inside a stage; X first so its chunks stay 1024-aligned)
   __host__ __device__ static constexpr int x_chunk(int mpad) { return mpad * 128; }
   __host__ __device__ static constexpr int stage_bytes(int mpad) {
@@ -60,7 +64,7 @@ struct W4Cfg {
   }
   __host__ __device__ static constexpr int bar_offset(int mpad) { return nst(mpad) * stage_bytes(mpad); }
   __host__ __device__ static constexpr int smem_bytes(int mpad) {
-    return bar_offset(mpad) + (2 * MAX_NST + 6) * 8 + 16 + 1024;
+    return bar_offset(mpad) + (2 * MAX_NST + 2 * MAX_NA + 2) * 8 + 16 + 1024;
   }
   // the largest smem_bytes over every M (the kernel attribute must cover all)
   __host__ static constexpr int max_smem_bytes() {
@@ -92,11 +96,13 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
   const int NST = C::nst(mpad);
   uint64_t* full = bars;                     // NST: TMA bytes
   uint64_t* empty = full + C::MAX_NST;       // NST: MMA commit (X read) + 4 dequant warps (words read)
-  uint64_t* a_full = empty + C::MAX_NST;     // 2: 4 dequant warps
-  uint64_t* a_empty = a_full + 2;            // 2: MMA commit
-  uint64_t* done = a_empty + 2;              // 1
+  const int NA = C::na(mpad);
+  const uint32_t T_D = C::t_d(mpad);
+  uint64_t* a_full = empty + C::MAX_NST;     // NA: 4 dequant warps
+  uint64_t* a_empty = a_full + C::MAX_NA;    // NA: MMA commit
+  uint64_t* done = a_empty + C::MAX_NA;      // 1
   uint64_t* drain_bar = done + 1;            // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::MAX_NST + 6);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::MAX_NST + 2 * C::MAX_NA + 2);
   uint32_t* abort_word = tmem_slot + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -113,7 +119,7 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
       mbar_init(full + s, 1);
       mbar_init(empty + s, 5);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NA; ++b) {
       mbar_init(a_full + b, 4);
       mbar_init(a_empty + b, 1);
     }
@@ -175,15 +181,15 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     constexpr uint32_t hi = smem_desc_hi(1024);
     const uint32_t x_lo = smem_desc_lo(smem_addr(smem), 16);
     for (int g = 0; g < G; ++g) {
-      const int s = g % NST, b = g & 1;
+      const int s = g % NST, b = g % NA;
       if (!(ok = wait_all(full + s, (g / NST) & 1))) break;
-      if (!(ok = wait_all(a_full + b, (g >> 1) & 1))) break;
+      if (!(ok = wait_all(a_full + b, (g / NA) & 1))) break;
       tc_fence_after();
       const uint32_t xa = x_lo + ((s * SB) >> 4);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * XC + (kk & 3) * 32) >> 4;
-        mma_f16_ts(tmem_base + C::T_D, tmem_base + C::T_A + 64 * b + 8 * kk, smem_desc(xa + off, hi), idesc,
+        mma_f16_ts(tmem_base + T_D, tmem_base + C::T_A + 64 * b + 8 * kk, smem_desc(xa + off, hi), idesc,
                    (g > 0 || kk > 0) ? 1u : 0u, leader);
       }
       mma_commit(empty + s, leader);
@@ -202,9 +208,9 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     const int t = wq * 32 + lane;                    // output column n0 + t, TMEM lane t
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     for (int g = 0; g < G; ++g) {
-      const int s = g % NST, b = g & 1;
+      const int s = g % NST, b = g % NA;
       if (!(ok = wait_all(full + s, (g / NST) & 1))) break;
-      if (g >= 2 && !(ok = wait_all(a_empty + b, ((g >> 1) - 1) & 1))) break;
+      if (g >= NA && !(ok = wait_all(a_empty + b, ((g / NA) - 1) & 1))) break;
       const __half2 ss = __half2half2(s_at(s)[t]);
       // 1024 + z as fp16: the unpacked words below hold 1024 + q (exponent bits
       // 0x6400 with q in the low mantissa bits), so one subtraction gives q - z exactly
@@ -238,7 +244,7 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
       __half* ycol = p.y + n0 + t;
       for (int c0 = 0; c0 < mpad; c0 += 16) {
         uint32_t v[16];
-        tmem_ld16(tmem_base + lane_off + C::T_D + c0, v);
+        tmem_ld16(tmem_base + lane_off + T_D + c0, v);
         tmem_ld_wait<16>(v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
