@@ -51,7 +51,15 @@ struct BwdCfg {
   static constexpr int CHUNKS = D / 64;
   static constexpr int TILE_BYTES = CHUNKS * CHUNK_BYTES;    // one 128-row tile of Q, K, V or dO
   static constexpr int NST = 2;                              // ring stages
-  static constexpr int THREADS = 256;
+  // compute warpgroups: with two, the two warps of a TMEM lane quarter split the
+  // 128 columns of each row (64 each), so each thread has half the exponentials
+  // and the latencies of one warp hide under the other's work
+#ifndef ATTN_BWD_SPLIT
+#define ATTN_BWD_SPLIT 2
+#endif
+  static constexpr int SPLIT = ATTN_BWD_SPLIT;
+  static constexpr int NCOL = 128 / SPLIT;                   // columns per compute thread
+  static constexpr int THREADS = 128 + 128 * SPLIT;
   static constexpr int COMPUTE_WARP0 = 4;
   static constexpr uint32_t TMEM_COLS = 512;
   // dkdv shared memory: K, V, then per stage {Q, dO, lse2[128], D[128]}
@@ -197,6 +205,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* ds_ready = p_ready + 1;         // 1 (4 compute warps)
   uint64_t* done = ds_ready + 1;            // 1
   uint64_t* drain_bar = done + 1;           // 1
+  uint64_t* s_read = drain_bar + 1;         // 1 (SPLIT 2: the first column half has read S^T)
+  uint64_t* dp_read = s_read + 1;           // 1 (SPLIT 2: the first column half has read dP^T)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   uint32_t* abort_word = tmem_slot + 1;
 
@@ -215,10 +225,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
-    mbar_init(p_ready, 4);
-    mbar_init(ds_ready, 4);
+    mbar_init(p_ready, 4 * C::SPLIT);
+    mbar_init(ds_ready, 4 * C::SPLIT);
     mbar_init(done, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(s_read, 4);
+    mbar_init(dp_read, 4);
     *abort_word = 0u;
     fence_barrier_init();
     fence_proxy_async_shared();
@@ -330,7 +342,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
   } else if (warp >= C::COMPUTE_WARP0) {
     // ======================= compute: one thread per key =======================
-    const int wq = warp - C::COMPUTE_WARP0;
+    // Thread (key r, column half h) owns the queries [NCOL h, NCOL h + NCOL) of its
+    // row. Packed bf16 P^T / dS^T of half h goes to the columns [NCOL h / 2, ...)
+    // of S^T / dP^T, which for h = 1 overlap columns half 0 reads: half 1 stores
+    // only after half 0 has read (s_read, dp_read).
+    constexpr int NCOL = C::NCOL;
+    const int cw = warp - C::COMPUTE_WARP0;
+    const int wq = warp & 3;                            // TMEM lane quarter of this warp
+    const int h = cw >> 2;                              // column half
+    const int col0 = NCOL * h;
     const int r = wq * 32 + lane;                       // key inside the block
     const int key = jb * 128 + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -343,34 +363,41 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (!(ok = wait_all(s_full, it & 1))) break;
       tc_fence_after();
       // the block's statistics are the same for every thread: 16-byte broadcast loads
-      const float4* lse2 = reinterpret_cast<const float4*>(stage_lse(s));
-      const float4* dd = reinterpret_cast<const float4*>(stage_dd(s));
-      float pr[128];
+      const float4* lse2 = reinterpret_cast<const float4*>(stage_lse(s) + col0);
+      const float4* dd = reinterpret_cast<const float4*>(stage_dd(s) + col0);
+      float pr[NCOL];
       {
-        uint32_t sr[128];
-        tmem_ld32(t_s + 0, sr + 0);
-        tmem_ld32(t_s + 32, sr + 32);
-        tmem_ld32(t_s + 64, sr + 64);
-        tmem_ld32(t_s + 96, sr + 96);
-        tmem_ld_wait<128>(sr);
+        uint32_t sr[NCOL];
+#pragma unroll
+        for (int q = 0; q < NCOL / 32; ++q) tmem_ld32(t_s + col0 + 32 * q, sr + 32 * q);
+        tmem_ld_wait<NCOL>(sr);
+        if (C::SPLIT > 1 && h == 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_read);
+        }
         // visible: key < N, and for the diagonal block of a causal launch, key <= query
         const int first_visible = (key >= p.N) ? 128 : ((p.causal && i == jb) ? r : 0);
 #pragma unroll
-        for (int j4 = 0; j4 < 32; ++j4) {
+        for (int j4 = 0; j4 < NCOL / 4; ++j4) {
           const float4 l4 = lse2[j4];
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int j = 4 * j4 + e;
             const float x = ex2_approx(fmaf(__uint_as_float(sr[j]), c, -lv[e]));
-            pr[j] = (j >= first_visible) ? x : 0.f;
+            pr[j] = (col0 + j >= first_visible) ? x : 0.f;
           }
         }
-        uint32_t pk[64];
+        uint32_t pk[NCOL / 2];
 #pragma unroll
-        for (int j = 0; j < 64; ++j) pk[j] = pack_bf16x2(pr[2 * j], pr[2 * j + 1]);
-        tmem_st32(t_s + 0, pk);
-        tmem_st32(t_s + 32, pk + 32);
+        for (int j = 0; j < NCOL / 2; ++j) pk[j] = pack_bf16x2(pr[2 * j], pr[2 * j + 1]);
+        if (C::SPLIT > 1 && h > 0) {
+          if (!(ok = wait_all(s_read, it & 1))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int q = 0; q < NCOL / 64; ++q) tmem_st32(t_s + col0 / 2 + 32 * q, pk + 32 * q);
         tmem_st_wait();
       }
       tc_fence_before();
@@ -378,11 +405,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (lane == 0) mbar_arrive(p_ready);
       if (!(ok = wait_all(dp_full, it & 1))) break;
       tc_fence_after();
+      bool first_store = true;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < NCOL / 32; ++ch) {
         uint32_t dp[32];
-        tmem_ld32(t_dp + 32 * ch, dp);
+        tmem_ld32(t_dp + col0 + 32 * ch, dp);
         tmem_ld_wait<32>(dp);
+        if (C::SPLIT > 1 && h == 0 && ch == NCOL / 32 - 1) {   // half 0 has read all its dP^T
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(dp_read);
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 16; j += 2) {
@@ -393,8 +426,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           pk[j + 1] = pack_bf16x2(pr[q0 + 2] * (__uint_as_float(dp[2 * j + 2]) - d4.z),
                                   pr[q0 + 3] * (__uint_as_float(dp[2 * j + 3]) - d4.w));
         }
-        tmem_st16(t_dp + 16 * ch, pk);   // dS^T over the dP^T columns already read
+        if (C::SPLIT > 1 && h > 0 && first_store) {
+          if (!(ok = wait_all(dp_read, it & 1))) break;
+          tc_fence_after();
+        }
+        first_store = false;
+        tmem_st16(t_dp + col0 / 2 + 16 * ch, pk);   // dS^T over dP^T columns already read
       }
+      if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -405,8 +444,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_fence_after();
       const bool in_range = key < p.N;
       const size_t row = static_cast<size_t>(bh) * p.N + (in_range ? key : 0);
-      store_row_bf16<C::D>(tmem_base + lane_off + C::T_DV, 1.f, p.dv + row * C::D, in_range);
-      store_row_bf16<C::D>(tmem_base + lane_off + C::T_DK, p.scale, p.dk + row * C::D, in_range);
+      if (C::SPLIT == 1 || h == 0)
+        store_row_bf16<C::D>(tmem_base + lane_off + C::T_DV, 1.f, p.dv + row * C::D, in_range);
+      if (C::SPLIT == 1 || h == 1)
+        store_row_bf16<C::D>(tmem_base + lane_off + C::T_DK, p.scale, p.dk + row * C::D, in_range);
     } else if (lane == 0) {
       record_timeout();
     }
@@ -433,9 +474,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* kv_empty = kv_full + C::NST;    // NST
   uint64_t* s_full = kv_empty + C::NST;     // 2 (S buffers)
   uint64_t* dp_full = s_full + 2;           // 1
-  uint64_t* ds_ready = dp_full + 1;         // 1 (4 compute warps)
+  uint64_t* ds_ready = dp_full + 1;         // 1 (all compute warps)
   uint64_t* done = ds_ready + 1;            // 1
   uint64_t* drain_bar = done + 1;           // 1
+  uint64_t* s_read = drain_bar + 1;         // 1 (SPLIT 2: the first column half has read S)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NUM_BARS);
   uint32_t* abort_word = tmem_slot + 1;
 
@@ -454,9 +496,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(s_full + 0, 1);
     mbar_init(s_full + 1, 1);
     mbar_init(dp_full, 1);
-    mbar_init(ds_ready, 4);
+    mbar_init(ds_ready, 4 * C::SPLIT);
     mbar_init(done, 1);
     mbar_init(drain_bar, 1);
+    mbar_init(s_read, 4);
     *abort_word = 0u;
     fence_barrier_init();
     fence_proxy_async_shared();
@@ -558,7 +601,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
   } else if (warp >= C::COMPUTE_WARP0) {
     // ======================= compute: one thread per query =======================
-    const int wq = warp - C::COMPUTE_WARP0;
+    // Thread (query r, column half h) owns the keys [NCOL h, NCOL h + NCOL) of its
+    // row; its packed bf16 dS goes to S columns [NCOL h / 2, ...), which for h = 1
+    // overlap columns half 0 reads: half 1 stores only after half 0 has read (s_read).
+    constexpr int NCOL = C::NCOL;
+    const int cw = warp - C::COMPUTE_WARP0;
+    const int wq = warp & 3;
+    const int h = cw >> 2;
+    const int col0 = NCOL * h;
     const int r = wq * 32 + lane;
     const int qrow = ib * 128 + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -570,28 +620,31 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const uint32_t t_s = tmem_base + lane_off + C::T_S + 128 * (j & 1);
       if (!(ok = wait_all(s_full + (j & 1), (j >> 1) & 1))) break;
       tc_fence_after();
-      float pr[128];
+      float pr[NCOL];
       {
-        uint32_t sr[128];
-        tmem_ld32(t_s + 0, sr + 0);
-        tmem_ld32(t_s + 32, sr + 32);
-        tmem_ld32(t_s + 64, sr + 64);
-        tmem_ld32(t_s + 96, sr + 96);
-        tmem_ld_wait<128>(sr);
+        uint32_t sr[NCOL];
+#pragma unroll
+        for (int q = 0; q < NCOL / 32; ++q) tmem_ld32(t_s + col0 + 32 * q, sr + 32 * q);
+        tmem_ld_wait<NCOL>(sr);
+        if (C::SPLIT > 1 && h == 0) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_read);
+        }
         // visible keys: j*128 + col < N and, on a causal diagonal block, col <= r
         int last = p.N - 1 - j * 128;
         if (p.causal && j == ib) last = min(last, r);
 #pragma unroll
-        for (int k = 0; k < 128; ++k) {
+        for (int k = 0; k < NCOL; ++k) {
           const float x = ex2_approx(fmaf(__uint_as_float(sr[k]), c, -l2));
-          pr[k] = (k <= last) ? x : 0.f;
+          pr[k] = (col0 + k <= last) ? x : 0.f;
         }
       }
       if (!(ok = wait_all(dp_full, j & 1))) break;
       tc_fence_after();
-      const uint32_t t_dp = tmem_base + lane_off + C::T_DPQ;
+      const uint32_t t_dp = tmem_base + lane_off + C::T_DPQ + col0;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int ch = 0; ch < NCOL / 32; ++ch) {
         uint32_t dp[32];
         tmem_ld32(t_dp + 32 * ch, dp);
         tmem_ld_wait<32>(dp);
@@ -601,8 +654,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           const int k0 = 32 * ch + 2 * k;
           pk[k] = pack_bf16x2(pr[k0] * (__uint_as_float(dp[2 * k]) - dd), pr[k0 + 1] * (__uint_as_float(dp[2 * k + 1]) - dd));
         }
-        tmem_st16(t_s + 16 * ch, pk);   // dS over the S columns already read
+        if (C::SPLIT > 1 && h > 0 && ch == 0) {
+          if (!(ok = wait_all(s_read, j & 1))) break;
+          tc_fence_after();
+        }
+        tmem_st16(t_s + col0 / 2 + 16 * ch, pk);   // dS over the S columns already read
       }
+      if (!ok) break;
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -612,7 +670,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (ok) {
       tc_fence_after();
       const bool in_range = qrow < p.N;
-      store_row_bf16<C::D>(tmem_base + lane_off + C::T_DQ, p.scale, p.dq + g * C::D, in_range);
+      // the two column halves of a row store the two halves of its dQ
+      constexpr int DC = C::D / C::SPLIT;
+      store_row_bf16<DC>(tmem_base + lane_off + C::T_DQ + DC * h, p.scale, p.dq + g * C::D + DC * h, in_range);
     } else if (lane == 0) {
       record_timeout();
     }
