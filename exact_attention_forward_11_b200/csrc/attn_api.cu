@@ -50,10 +50,53 @@ constexpr uint64_t kWaitLimitCycles = 1ull << 31;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Encoded maps are kept in a small cache keyed by everything the encoding
+// depends on (a map is a pure function of base address, type and shape), so a
+// caller that repeats a call on the same buffers skips the host-side encoding.
+struct MapKey {
+  const void* base;
+  int fp8, d, N, BH, rows;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && fp8 == o.fp8 && d == o.d && N == o.N && BH == o.BH && rows == o.rows;
+  }
+};
+constexpr int kMapCacheSize = 32;
+struct MapCache {
+  std::mutex mu;
+  MapKey key[kMapCacheSize];
+  CUtensorMap map[kMapCacheSize];
+  int used = 0, next = 0;
+};
+MapCache& map_cache() {
+  static MapCache c;
+  return c;
+}
+
+bool encode_qkv_map_uncached(CUtensorMap* map, const void* base, bool fp8, int d, int N, int BH, int rows);
+
 // 3-D map over a contiguous [BH, N, d] tensor: dims {d, N, BH}, box {128 bytes of
 // d, `rows` rows, 1}, 128-byte swizzle (the layout the MMA descriptors expect).
 // Rows past N read as zero.
 bool encode_qkv_map(CUtensorMap* map, const void* base, bool fp8, int d, int N, int BH, int rows) {
+  const MapKey k{base, fp8 ? 1 : 0, d, N, BH, rows};
+  MapCache& c = map_cache();
+  {
+    std::lock_guard<std::mutex> lock(c.mu);
+    for (int i = 0; i < c.used; ++i)
+      if (c.key[i] == k) {
+        *map = c.map[i];
+        return true;
+      }
+  }
+  if (!encode_qkv_map_uncached(map, base, fp8, d, N, BH, rows)) return false;
+  std::lock_guard<std::mutex> lock(c.mu);
+  const int slot = c.used < kMapCacheSize ? c.used++ : (c.next++ % kMapCacheSize);
+  c.key[slot] = k;
+  c.map[slot] = *map;
+  return true;
+}
+
+bool encode_qkv_map_uncached(CUtensorMap* map, const void* base, bool fp8, int d, int N, int BH, int rows) {
   EncodeTiledFn enc = get_encode_fn();
   if (enc == nullptr) return false;
   const int elem = fp8 ? 1 : 2;

@@ -19,9 +19,11 @@
 // per output column = one TMEM lane, tcgen05.st) and are the MMA's A operand
 // from TMEM; only the small X slice is read from shared memory by the MMA.
 //
-// CTA: 8 warps. warp 0 TMA producer (weight words, scales, zero points and the X
-// slice of each K slice into a ring of up to 8 stages), warp 1 MMA issuer (owns TMEM),
-// warps 2-3 idle, warps 4-7 dequantise (thread t: column n0 + t) and write Y.
+// CTA: 12 warps. warp 0 TMA producer (weight words, scales, zero points and the X
+// slice of each K slice into a ring of up to 8 stages), warp 1 MMA issuer (owns
+// TMEM), warps 2-3 idle, warps 4-11 dequantise (thread t of quarter q: column
+// n0 + 32 q + t; warps 4-7 take the first 8 words of a slice, 8-11 the last 8)
+// and warps 4-7 write Y. Two CTAs fit on an SM (85 registers per thread).
 // TMEM: three (two for M > 64) 64-column A buffers (a 128-deep slice of fp16
 // pairs each) and the MPAD-column fp32 accumulator. Every wait is bounded (Waiter).
 #pragma once
@@ -36,7 +38,15 @@
 namespace attn {
 
 struct W4Cfg {
-  static constexpr int THREADS = 256;
+  // dequantisation warpgroups: with two, the two warps of a TMEM lane quarter
+  // each unpack half of a slice's words (64 of its 128 k), so one warp's TMEM
+  // store and wait overlap the other's unpacking
+#ifndef ATTN_W4_SPLIT
+#define ATTN_W4_SPLIT 2
+#endif
+  static constexpr int SPLIT = ATTN_W4_SPLIT;
+  static constexpr int WORDS = 16 / SPLIT;     // packed words per thread per slice
+  static constexpr int THREADS = 128 + 128 * SPLIT;
   static constexpr int MAX_NST = 8;            // ring stages: as many as ~110 KB of shared memory holds
   static constexpr int GROUP = 128;            // k per scale / zero point = k per slice
   static constexpr int BN = 128;               // output columns per CTA
@@ -81,7 +91,7 @@ struct W4Params {
   uint64_t timeout_cycles;
 };
 
-__global__ void __launch_bounds__(W4Cfg::THREADS, 1)
+__global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     w4a16_gemm_sm100(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                      const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z,
                      const W4Params p) {
@@ -117,10 +127,10 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, 5);
+      mbar_init(empty + s, 1 + 4 * C::SPLIT);
     }
     for (int b = 0; b < NA; ++b) {
-      mbar_init(a_full + b, 4);
+      mbar_init(a_full + b, 4 * C::SPLIT);
       mbar_init(a_empty + b, 1);
     }
     mbar_init(done, 1);
@@ -204,7 +214,8 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ======================= dequantise, then Y =======================
-    const int wq = warp - 4;
+    const int wq = warp & 3;                         // TMEM lane quarter
+    const int h = (warp - 4) >> 2;                   // which words of the slice (SPLIT 2)
     const int t = wq * 32 + lane;                    // output column n0 + t, TMEM lane t
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     for (int g = 0; g < G; ++g) {
@@ -217,10 +228,10 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
       const __half zh = __ushort_as_half(static_cast<unsigned short>(0x6400u | z_at(s)[t]));
       const __half2 zz = __half2half2(zh);
       const uint32_t* wrow = w_at(s);
-      uint32_t pk[64];
+      uint32_t pk[4 * C::WORDS];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const uint32_t word = wrow[i * C::BN + t];
+      for (int i = 0; i < C::WORDS; ++i) {
+        const uint32_t word = wrow[(C::WORDS * h + i) * C::BN + t];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           // bits 4j..4j+3 (weight 8i+2j) into the low half, bits 16+4j.. (8i+2j+1) into the high half
@@ -231,15 +242,17 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty + s);         // this warp's words, scale and zero are read
-      tmem_st32(tmem_base + lane_off + C::T_A + 64 * b, pk);
-      tmem_st32(tmem_base + lane_off + C::T_A + 64 * b + 32, pk + 32);
+#pragma unroll
+      for (int q = 0; q < C::WORDS / 8; ++q)
+        tmem_st32(tmem_base + lane_off + C::T_A + 64 * b + 4 * C::WORDS * h + 32 * q, pk + 32 * q);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(a_full + b);
     }
-    if (ok) ok = wait_all(done, 0);
-    if (ok) {
+    // Y: the first warpgroup reads the accumulator and writes the tile
+    if (ok && h == 0) ok = wait_all(done, 0);
+    if (ok && h == 0) {
       tc_fence_after();
       __half* ycol = p.y + n0 + t;
       for (int c0 = 0; c0 < mpad; c0 += 16) {
