@@ -54,28 +54,38 @@ def gather_heads(local, BH: int, group=None):
     return torch.cat(parts, dim=0)
 
 
-def forward_sharded(q, k, v, causal=False, scale=None, group=None, with_lse=True, stream=None):
-    """O, LSE of attention over q, k, v [B, H, N, d] (bf16 CUDA, the same on every
-    rank), computed head-sharded: this rank runs attn_fwd on its own heads only,
-    then one all-gather gives every rank the full O [B, H, N, d] and LSE [B, H, N]."""
+def forward_heads(q, k, v, start, count, causal=False, scale=None, stream=None):
+    """O [count, N, d] and LSE [count, N] of the heads [start, start + count) of the
+    flattened B*H axis, computed by attn_fwd on pointer offsets into q, k, v (no copy)."""
     import torch
-    import torch.distributed as dist
 
     from . import _check, _expect, _shape4, _stream_ptr, attn_fwd, ATTN_BF16
     B, H, N, d = _shape4(q)
     for name, t in (("q", q), ("k", k), ("v", v)):
         _expect(t, name, (B, H, N, d), torch.bfloat16, q.device)
-    BH = B * H
-    world, rank = dist.get_world_size(group), dist.get_rank(group)
-    start, cnt = head_range(BH, world, rank)
-    o_loc = torch.empty((cnt, N, d), dtype=torch.bfloat16, device=q.device)
-    l_loc = torch.empty((cnt, N), dtype=torch.float32, device=q.device)
-    if cnt > 0:
+    if start < 0 or count < 0 or start + count > B * H:
+        raise ValueError("head range outside the tensor")
+    o_loc = torch.empty((count, N, d), dtype=torch.bfloat16, device=q.device)
+    l_loc = torch.empty((count, N), dtype=torch.float32, device=q.device)
+    if count > 0:
         off = start * N * d * q.element_size()
         sc = 0.0 if scale is None else float(scale)
         _check(attn_fwd(q.data_ptr() + off, k.data_ptr() + off, v.data_ptr() + off, o_loc.data_ptr(),
-                        l_loc.data_ptr() if with_lse else None, 1, cnt, N, d, sc, int(bool(causal)), ATTN_BF16,
+                        l_loc.data_ptr(), 1, count, N, d, sc, int(bool(causal)), ATTN_BF16,
                         _stream_ptr(q, stream)), "attn_fwd")
+    return o_loc, l_loc
+
+
+def forward_sharded(q, k, v, causal=False, scale=None, group=None, stream=None):
+    """O, LSE of attention over q, k, v [B, H, N, d] (bf16 CUDA, the same on every
+    rank), computed head-sharded: this rank runs attn_fwd on its own heads only,
+    then one all-gather gives every rank the full O [B, H, N, d] and LSE [B, H, N]."""
+    import torch.distributed as dist
+    B, H, N, d = q.shape
+    BH = B * H
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    start, cnt = head_range(BH, world, rank)
+    o_loc, l_loc = forward_heads(q, k, v, start, cnt, causal=causal, scale=scale, stream=stream)
     o = gather_heads(o_loc, BH, group).view(B, H, N, d)
-    lse = gather_heads(l_loc, BH, group).view(B, H, N) if with_lse else None
+    lse = gather_heads(l_loc, BH, group).view(B, H, N)
     return o, lse
