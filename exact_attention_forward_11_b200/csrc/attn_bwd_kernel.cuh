@@ -212,8 +212,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int QB = (p.N + 127) / 128;
-  const int jb = blockIdx.x / p.BH;                 // key block (heaviest causal blocks first)
-  const int bh = blockIdx.x % p.BH;
+  // CTA -> (key block, head). Head-major order keeps the CTAs that run together
+  // on a few heads, whose Q / dO tiles they all stream, so those come from L2;
+  // inside a head the heaviest causal key blocks go first.
+#ifndef ATTN_BWD_HEAD_MAJOR
+#define ATTN_BWD_HEAD_MAJOR 1
+#endif
+  const int jb = ATTN_BWD_HEAD_MAJOR ? static_cast<int>(blockIdx.x) % QB : static_cast<int>(blockIdx.x) / p.BH;
+  const int bh = ATTN_BWD_HEAD_MAJOR ? static_cast<int>(blockIdx.x) / QB : static_cast<int>(blockIdx.x) % p.BH;
   const int i0 = p.causal ? jb : 0;                 // first visible query block
   const int n = QB - i0;                            // query blocks visited
 
@@ -483,8 +489,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int QB = (p.N + 127) / 128;
-  const int ib = QB - 1 - static_cast<int>(blockIdx.x) / p.BH;   // query block (heaviest causal first)
-  const int bh = blockIdx.x % p.BH;
+  // CTA -> (query block, head): head-major (the K / V tiles of the CTAs running
+  // together come from L2), heaviest causal query blocks first inside a head
+  const int ib = QB - 1 - (ATTN_BWD_HEAD_MAJOR ? static_cast<int>(blockIdx.x) % QB
+                                               : static_cast<int>(blockIdx.x) / p.BH);
+  const int bh = ATTN_BWD_HEAD_MAJOR ? static_cast<int>(blockIdx.x) / QB : static_cast<int>(blockIdx.x) % p.BH;
   const int n = p.causal ? ib + 1 : QB;                          // key blocks visited
 
   if (threadIdx.x == 0) {

@@ -252,7 +252,9 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     }
     // Y: the first warpgroup reads the accumulator and writes the tile
     if (ok && h == 0) ok = wait_all(done, 0);
-    if (ok && h == 0) {
+    if (!ok) {
+      if (lane == 0) record_timeout();
+    } else if (h == 0) {
       tc_fence_after();
       __half* ycol = p.y + n0 + t;
       for (int c0 = 0; c0 < mpad; c0 += 16) {
@@ -265,8 +267,6 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
           if (m < p.M) ycol[static_cast<size_t>(m) * p.N] = __float2half_rn(__uint_as_float(v[i]));
         }
       }
-    } else if (lane == 0) {
-      record_timeout();
     }
   }
 
