@@ -2,8 +2,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-One step = one full pass of the hot path (one attn_fwd launch, or for the FP8
-workload the three preparation launches plus attn_fwd_fp8) over one batch of
+One step = one full pass of the hot path (one attn_fwd launch; for the FP8
+workload the three preparation launches plus attn_fwd_fp8; for the MXFP8 workload
+the three attn_quantize_mxfp8 launches plus attn_fwd_mxfp8) over one batch of
 synthetic inputs already resident in HBM. The default workload is the LLM
 training shape B=4, H=32, N=4096, d=128, causal, bf16: its inputs (403 MB) are
 larger than L2 (126 MB), so no L2 flush is needed between timed iterations.
@@ -32,7 +33,7 @@ sys.path.insert(0, HERE)
 
 import workloads  # noqa: E402
 
-METRIC = "attention fwd TFLOPS (BF16 / FP8) and % of B200 tensor-core peak"
+METRIC = "attention fwd TFLOPS (BF16 / FP8 / MXFP8) and % of B200 tensor-core peak"
 METRIC_BWD = "attention bwd TFLOPS (BF16, 2.5x forward FLOPs) and % of B200 tensor-core peak"
 METRIC_W4A16 = "W4A16 GEMM TFLOPS (fp16 activations, int4 weights dequantised on the fly) and % of HBM roofline"
 DEFAULT_WORKLOAD = "llm_train_causal"
@@ -275,7 +276,7 @@ class Step:
         import torch
         self.lib, self.w = lib, w
         self.dev = dev
-        self.copies = 1 if w.fp8 else l2_copies(w)
+        self.copies = 1 if (w.fp8 or w.mx) else l2_copies(w)
         self.sets = []
         for c in range(self.copies):
             qkv = [x[n].to(dev) if c == 0 else x[n].to(dev).clone() for n in ("q", "k", "v")]
@@ -289,9 +290,13 @@ class Step:
             T = (w.N + 127) // 128
             self.codes = [torch.empty((w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8) for _ in range(3)]
             self.scales = [torch.empty((w.B, w.H, T), device=dev, dtype=torch.float32) for _ in range(3)]
-        self.launches = 4 if w.fp8 else 1
+        if w.mx:
+            self.codes = [torch.empty((w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8) for _ in range(3)]
+            self.sfs = [torch.empty((w.B, w.H, w.N, w.d // 32), device=dev, dtype=torch.uint8) for _ in range(3)]
+        self.launches = 4 if (w.fp8 or w.mx) else 1
+        self.attn_kernel = "attn_fwd1_sm100" if w.mx else "attn_fwd_sm100"
         self.kernels = (["fp8_rotate_quantize", "fp8_quantize", "attn_fwd_sm100"] if w.fp8
-                        else ["attn_fwd_sm100"])
+                        else ["mxfp8_quantize", "attn_fwd1_sm100"] if w.mx else ["attn_fwd_sm100"])
 
     def run_device(self, stream, mark=None):
         """Launches one step on `stream`; mark(kernel name), if given, is called
@@ -299,6 +304,19 @@ class Step:
         lib, w = self.lib, self.w
         s = stream.cuda_stream
         mark = mark or (lambda name: None)
+        if w.mx:
+            for src, c8, sf in zip((self.q, self.k, self.v), self.codes, self.sfs):
+                st = lib.attn_quantize_mxfp8(src.data_ptr(), c8.data_ptr(), sf.data_ptr(), w.B, w.H, w.N, w.d, s)
+                if st:
+                    raise lib.AttnError(st, "attn_quantize_mxfp8")
+                mark("mxfp8_quantize")
+            st = lib.attn_fwd_mxfp8(*(c.data_ptr() for c in self.codes), *(f.data_ptr() for f in self.sfs),
+                                    self.o.data_ptr(), self.lse.data_ptr(), w.B, w.H, w.N, w.d, w.scale,
+                                    int(w.causal), s)
+            if st:
+                raise lib.AttnError(st, "attn_fwd_mxfp8")
+            mark("attn_fwd1_sm100")
+            return
         if not w.fp8:
             q, k, v, o, lse = self.sets[self.i]
             self.i = (self.i + 1) % self.copies
@@ -557,6 +575,11 @@ def time_e2e(lib, w, x, dev, stream, steps):
                 k8, ks = lib.quantize_fp8(dk, extra["rot"], stream=stream)
                 v8, vs = lib.quantize_fp8(dv, None, stream=stream)
                 lib.forward_fp8(q8, k8, v8, qs, ks, vs, causal=w.causal, out=do, lse=dl, stream=stream)
+            elif w.mx:
+                q8, qs = lib.quantize_mxfp8(dq, stream=stream)
+                k8, ks = lib.quantize_mxfp8(dk, stream=stream)
+                v8, vs = lib.quantize_mxfp8(dv, stream=stream)
+                lib.forward_mxfp8(q8, k8, v8, qs, ks, vs, causal=w.causal, out=do, lse=dl, stream=stream)
             else:
                 lib.forward(dq, dk, dv, causal=w.causal, out=do, lse=dl, stream=stream)
             o_host.copy_(do, non_blocking=True)
@@ -594,12 +617,22 @@ def prep_bytes(w):
     return w.B * w.H * w.N * w.d * 3 + 4 * w.B * w.H * T
 
 
-def roofline(w, kern_ms, sm_mhz, workload):
+def mx_prep_bytes(w):
+    """Algorithmic bytes of one MXFP8 quantisation launch: bf16 read, one code byte
+    and 1/32 scale byte written per element."""
+    n = w.B * w.H * w.N * w.d
+    return 2 * n + n + n // 32
+
+
+def roofline(w, kern_ms, sm_mhz, workload, kernel="attn_fwd_sm100"):
     """Roofline object of the dominant kernel (the attention kernel), from its
-    mean launch time measured with CUDA events in the timed loop."""
+    mean launch time measured with CUDA events in the timed loop. The MXFP8
+    attention kernel's S products run at the E4M3 rate and its P V products at
+    the 16-bit rate, so its denominator is the bf16 peak x 4/3 (the time the
+    tensor pipe needs for both products at those rates)."""
     peak_bf16, hbm, peak_src = measured_peaks()
     dt = "fp8" if w.fp8 else "bf16"
-    k_ms = kern_ms["attn_fwd_sm100"]
+    k_ms = kern_ms[kernel]
     if w.N < 1024 and not w.fp8:
         # small N (ViT shapes): arithmetic intensity below the ridge point, so the
         # roofline is HBM: algorithmic bytes = Q, K, V read once + O written (bf16) + LSE (fp32)
@@ -610,22 +643,25 @@ def roofline(w, kern_ms, sm_mhz, workload):
                 "peak_source": f"{peak_src} copy bandwidth", "kernel": "attn_fwd_sm100",
                 "algorithmic_bytes": bytes_launch, "kernel_ms": round(k_ms, 5)}
     achieved = w.flops / (k_ms * 1e-3) / 1e12
-    peak = peak_bf16 * (2 if w.fp8 else 1)
+    ratio = 2.0 if w.fp8 else (4.0 / 3.0 if w.mx else 1.0)
+    peak = round(peak_bf16 * ratio, 1)
+    note = {2.0: " x2 (fp8 nominal ratio)", 1.0: ""}.get(ratio, " x4/3 (E4M3 S at 2x, f16 P V at 1x the bf16 rate)")
     roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4), "traffic": traffic_per_launch(workload),
-            "peak_source": f"{peak_src} bf16 burst" + (" x2 (fp8 nominal ratio)" if w.fp8 else ""),
-            "kernel": "attn_fwd_sm100", "algorithmic_flops": w.flops, "kernel_ms": round(k_ms, 5),
-            "datasheet_peak": DATASHEET_TFLOPS[dt],
-            "frac_of_datasheet_peak": round(achieved / DATASHEET_TFLOPS[dt], 4)}
-    hw = hw_peak_tflops(dt, sm_mhz)
+            "peak_source": f"{peak_src} bf16 burst" + note,
+            "kernel": kernel, "algorithmic_flops": w.flops, "kernel_ms": round(k_ms, 5),
+            "datasheet_peak": round(DATASHEET_TFLOPS["bf16"] * ratio, 1),
+            "frac_of_datasheet_peak": round(achieved / (DATASHEET_TFLOPS["bf16"] * ratio), 4)}
+    hw = hw_peak_tflops("bf16", sm_mhz)
     if hw:
+        hw *= ratio
         roof["hw_peak_at_sampled_clock"] = round(hw, 1)
         roof["frac_of_hw_peak_at_sampled_clock"] = round(achieved / hw, 4)
     sus = sustained_bf16_peak()
     if sus:
         # a long timed loop meets the 1 kW power cap (see "clocks"); the sustained
         # GEMM rate is the same-conditions denominator
-        sus = sus * 2 if w.fp8 else sus
+        sus = round(sus * ratio, 1)
         roof["frac_of_sustained_peak"] = round(achieved / sus, 4)
         roof["sustained_peak"] = sus
     if w.fp8:
@@ -634,6 +670,12 @@ def roofline(w, kern_ms, sm_mhz, workload):
                                "gbs": round(pb / (kern_ms[name] * 1e-3) / 1e9, 1),
                                "frac_of_hbm": round(pb / (kern_ms[name] * 1e-3) / 1e9 / hbm, 4)}
                         for name in ("fp8_rotate_quantize", "fp8_quantize") if name in kern_ms}
+    if w.mx and "mxfp8_quantize" in kern_ms:
+        pb = mx_prep_bytes(w)
+        ms = kern_ms["mxfp8_quantize"]
+        roof["prep"] = {"mxfp8_quantize": {"ms": round(ms, 5), "algorithmic_bytes": pb,
+                                           "gbs": round(pb / (ms * 1e-3) / 1e9, 1),
+                                           "frac_of_hbm": round(pb / (ms * 1e-3) / 1e9 / hbm, 4)}}
     return roof
 
 
@@ -705,7 +747,7 @@ def run_ours(args):
     if w.fp8:
         x["rot64"], x["rot"] = workloads.make_rotation(w.d, w.seed + 7919)
     stream = torch.cuda.Stream(dev)
-    if args.bwd and w.fp8:
+    if args.bwd and (w.fp8 or w.mx):
         raise SystemExit("--bwd needs a BF16 workload")
     step = BwdStep(lib, w, x, dev) if args.bwd else Step(lib, w, x, dev)
     with ClockSampler(gpu_smi_id(dev, local)) as clk:
@@ -731,7 +773,7 @@ def run_ours(args):
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
     dt = "fp8" if w.fp8 else "bf16"
     roof = (roofline_bwd(w, kern_ms, clocks.get("sm_mhz")) if args.bwd
-            else roofline(w, kern_ms, clocks.get("sm_mhz"), args.workload))
+            else roofline(w, kern_ms, clocks.get("sm_mhz"), args.workload, step.attn_kernel))
     if w.fp8:
         roof["measured_fp8_gemm_burst_tflops"] = fp8_gemm_burst_tflops(dev)
     cpu = None
@@ -742,7 +784,8 @@ def run_ours(args):
     line = {
         "metric": METRIC_BWD if args.bwd else METRIC, "value": round(tflops, 3), "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3" if w.fp8 else "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3" if w.fp8 else ("mxfp8_e4m3_e8m0" if w.mx else "bf16"), "data": "synthetic",
         "config": {"workload": w.name, "B": w.B * world, "B_per_gpu": w.B, "H": w.H, "N": w.N, "d": w.d,
                    "causal": w.causal, "flops_per_step_per_gpu": flops_rank,
                    "pass": "backward" if args.bwd else "forward",
@@ -753,7 +796,8 @@ def run_ours(args):
         # the step's throughput against the datasheet dense tensor-core peak of the step's type
         "pct_of_peak": round(100 * tflops / world / DATASHEET_TFLOPS[dt], 2),
         "pct_of_peak_basis": f"B200 datasheet dense {dt.upper()} {DATASHEET_TFLOPS[dt]:.0f} TFLOP/s",
-        "pct_of_measured_peak": round(100 * tflops / world / (measured_peaks()[0] * (2 if w.fp8 else 1)), 2),
+        "pct_of_measured_peak": round(100 * tflops / world / (measured_peaks()[0] *
+                                                              (2 if w.fp8 else (4 / 3 if w.mx else 1))), 2),
         "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": step.launches * args.steps,
         "kernel_ms": {k: round(v, 5) for k, v in kern_ms.items()},
         "cycles_per_step": None if mhz is None else round(ms_step * 1e-3 * mhz * 1e6),
@@ -792,6 +836,16 @@ def oracle_sample(w, rows_per_head, heads, seed):
     else:
         fl = 4.0 * w.N * w.d * len(rows) * H
     from oracle import attention_fp64
+
+    if w.mx:
+        # the MXFP8 oracle: quantise and dequantise the sampled heads, then attend
+        from oracle.mxfp8 import mx_dequantize, mx_quantize
+
+        def call():
+            qd, kd, vd = (mx_dequantize(*mx_quantize(t)) for t in (q, k, v))
+            return attention_fp64(qd, kd, vd, w.scale, w.causal, rows=rows)
+        return call, fl, (f"{H} head(s) x {len(rows)} query rows of {w.name} (N={w.N}, d={w.d}), "
+                          f"MXFP8 quantisation of the sampled heads included")
 
     def call():
         return attention_fp64(q, k, v, w.scale, w.causal, rows=rows)

@@ -3,7 +3,8 @@
 The entry points below have the names and arguments of include/attn_b200.h and
 only marshal arguments: every step of the computation runs in the CUDA kernels
 of libattn_b200.so. There is no CPU fallback; if the library is missing the
-calls raise. `forward`, `quantize_fp8` and `forward_fp8` are torch conveniences
+calls raise. `forward`, `quantize_fp8`, `forward_fp8`, `quantize_mxfp8`, `forward_mxfp8`,
+`backward` and `w4a16_matmul` are torch conveniences
 that allocate outputs with torch (PyTorch serves only for device memory and
 streams) and call the same entry points.
 """
@@ -28,6 +29,8 @@ SIGNATURES = {
     "attn_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, _P]),
     "attn_quantize_fp8": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
     "attn_fwd_fp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "attn_quantize_mxfp8": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "attn_fwd_mxfp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_fwd_inject_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, ctypes.c_ulonglong, _P]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
@@ -71,6 +74,14 @@ def attn_quantize_fp8(x, rot, x8, scales, B, H, N, d, stream):
 
 def attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, scale, causal, stream):
     return load().attn_fwd_fp8(q8, k8, v8, q_scale, k_scale, v_scale, o, lse, B, H, N, d, scale, causal, stream)
+
+
+def attn_quantize_mxfp8(x, codes, sf, B, H, N, d, stream):
+    return load().attn_quantize_mxfp8(x, codes, sf, B, H, N, d, stream)
+
+
+def attn_fwd_mxfp8(q8, k8, v8, q_sf, k_sf, v_sf, o, lse, B, H, N, d, scale, causal, stream):
+    return load().attn_fwd_mxfp8(q8, k8, v8, q_sf, k_sf, v_sf, o, lse, B, H, N, d, scale, causal, stream)
 
 
 def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, B, H, N, d, scale, causal, stream):
@@ -221,6 +232,51 @@ def forward_fp8(q8, k8, v8, q_scale, k_scale, v_scale, causal=False, scale=None,
                         v_scale.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc, int(bool(causal)), sp),
            "attn_fwd_fp8")
     _check_device(check, sp, "attn_fwd_fp8")
+    return out, lse
+
+
+def quantize_mxfp8(x, stream=None):
+    """(codes uint8 [B,H,N,d], scale bytes uint8 [B,H,N,d/32]) of a bf16 tensor:
+    MXFP8, one E8M0 scale per 32 consecutive values of a row."""
+    import torch
+    B, H, N, d = _shape4(x)
+    _expect(x, "x", (B, H, N, d), torch.bfloat16, x.device)
+    codes = torch.empty((B, H, N, d), device=x.device, dtype=torch.uint8)
+    # the scale array is padded to 16 bytes so that its base stays 16-byte aligned
+    nsf = B * H * N * (d // 32)
+    sf = torch.empty(((nsf + 15) // 16) * 16, device=x.device, dtype=torch.uint8)[:nsf].view(B, H, N, d // 32)
+    _check(attn_quantize_mxfp8(x.data_ptr(), codes.data_ptr(), sf.data_ptr(), B, H, N, d, _stream_ptr(x, stream)),
+           "attn_quantize_mxfp8")
+    return codes, sf
+
+
+def forward_mxfp8(q8, k8, v8, q_sf, k_sf, v_sf, causal=False, scale=None, out=None, lse=None, with_lse=True,
+                  stream=None, check=False):
+    """O (bf16), LSE from MXFP8 codes [B,H,N,d] and their scale bytes [B,H,N,d/32].
+
+    Asynchronous like forward(): the outputs are valid once the launch has
+    finished and attn_get_device_status() reports ATTN_OK; check=True does both."""
+    import torch
+    B, H, N, d = _shape4(q8)
+    for name, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _expect(t, name, (B, H, N, d), torch.uint8, q8.device)
+    if d % 32:
+        raise ValueError("d must be a multiple of 32")
+    for name, t in (("q_sf", q_sf), ("k_sf", k_sf), ("v_sf", v_sf)):
+        _expect(t, name, (B, H, N, d // 32), torch.uint8, q8.device)
+    if out is None:
+        out = torch.empty((B, H, N, d), device=q8.device, dtype=torch.bfloat16)
+    _expect(out, "out", (B, H, N, d), torch.bfloat16, q8.device)
+    if lse is None and with_lse:
+        lse = torch.empty((B, H, N), device=q8.device, dtype=torch.float32)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, N), torch.float32, q8.device)
+    sc = 0.0 if scale is None else float(scale)
+    sp = _stream_ptr(q8, stream)
+    _check(attn_fwd_mxfp8(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), q_sf.data_ptr(), k_sf.data_ptr(),
+                          v_sf.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc, int(bool(causal)), sp),
+           "attn_fwd_mxfp8")
+    _check_device(check, sp, "attn_fwd_mxfp8")
     return out, lse
 
 

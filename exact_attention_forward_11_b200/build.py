@@ -16,7 +16,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libattn_b200.so")
 
 SOURCES = ["attn_api.cu"]
-HEADERS = ["sm100.cuh", "status.cuh", "attn_fwd_kernel.cuh", "attn_bwd_kernel.cuh", "fp8_prep_kernel.cuh", "w4a16_kernel.cuh"]
+HEADERS = ["sm100.cuh", "status.cuh", "attn_fwd_kernel.cuh", "attn_fwd1_kernel.cuh", "mxfp8_quant_kernel.cuh", "attn_bwd_kernel.cuh", "fp8_prep_kernel.cuh", "w4a16_kernel.cuh"]
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17",

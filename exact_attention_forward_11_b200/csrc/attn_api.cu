@@ -15,8 +15,10 @@
 #include "attn_b200_testing.h"
 #include "w4a16_b200.h"
 #include "attn_bwd_kernel.cuh"
+#include "attn_fwd1_kernel.cuh"
 #include "attn_fwd_kernel.cuh"
 #include "fp8_prep_kernel.cuh"
+#include "mxfp8_quant_kernel.cuh"
 #include "w4a16_kernel.cuh"
 
 // Scratch of attn_bwd_noalloc (D_i, 4 bytes per row) for at most
@@ -179,6 +181,21 @@ attn_status check_shape(int B, int H, int N) {
   return ATTN_OK;
 }
 
+// Non-causal: heads per group such that the group's K and V (2 N d elements per
+// head) take about 48 MB of the 126 MB L2. Causal: all heads unless
+// ATTN_CAUSAL_GROUP_MB gives a budget for causal groups too.
+#ifndef ATTN_CAUSAL_GROUP_MB
+#define ATTN_CAUSAL_GROUP_MB 0
+#endif
+int heads_per_group(int BH, int N, int D, int elem, int causal) {
+  const long long kv_bytes = 2ll * N * D * elem;
+  const long long budget = causal ? (static_cast<long long>(ATTN_CAUSAL_GROUP_MB) << 20) : (48ll << 20);
+  long long hg = budget == 0 ? BH : budget / (kv_bytes > 0 ? kv_bytes : 1);
+  if (hg < 1) hg = 1;
+  if (hg > BH) hg = BH;
+  return static_cast<int>(hg);
+}
+
 template <int D, bool FP8>
 attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const float* qs,
                        const float* ks, const float* vs, int BH, int N, float scale, int causal,
@@ -196,20 +213,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.N = N;
   p.BH = BH;
   p.num_units = BH * npair;
-  // Non-causal: heads per group such that the group's K and V (2 N d bytes per
-  // element per head) take about 48 MB of the 126 MB L2. Causal: all heads
-  // unless ATTN_CAUSAL_GROUP_MB gives a budget for causal groups too.
-#ifndef ATTN_CAUSAL_GROUP_MB
-#define ATTN_CAUSAL_GROUP_MB 0
-#endif
-  {
-    const long long kv_bytes = 2ll * N * C::D * (C::FP8 ? 1 : 2);
-    const long long budget = causal ? (static_cast<long long>(ATTN_CAUSAL_GROUP_MB) << 20) : (48ll << 20);
-    long long hg = budget == 0 ? BH : budget / (kv_bytes > 0 ? kv_bytes : 1);
-    if (hg < 1) hg = 1;
-    if (hg > BH) hg = BH;
-    p.heads_per_group = static_cast<int>(hg);
-  }
+  p.heads_per_group = heads_per_group(BH, N, C::D, C::FP8 ? 1 : 2, causal);
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -227,6 +231,44 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) {
     forget_smem(fwd_tag<D, FP8>());
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+// The one-Q-tile forward (attn_fwd1_kernel.cuh): BF16 (MX = false) or MXFP8
+// codes with their scale-byte arrays (MX = true).
+template <int D, bool MX>
+attn_status launch_fwd1(const void* q, const void* k, const void* v, void* o, float* lse, const void* q_sf,
+                        const void* k_sf, const void* v_sf, int BH, int N, float scale, int causal,
+                        cudaStream_t stream) {
+  using C = attn::Fwd1Cfg<D, MX>;
+  auto kern = attn::attn_fwd1_sm100<C>;
+  const int tag = MX ? 12 : (D == 128 ? 10 : 11);
+  CUtensorMap tq, tk, tv;
+  if (!encode_qkv_map(&tq, q, MX, D, N, BH, attn::kBlockM) || !encode_qkv_map(&tk, k, MX, D, N, BH, attn::kBlockN) ||
+      !encode_qkv_map(&tv, v, MX, D, N, BH, attn::kBlockN))
+    return ATTN_ERR_CUDA;
+  if (!set_smem_once(reinterpret_cast<const void*>(kern), C::SMEM_BYTES, tag)) return ATTN_ERR_CUDA;
+  attn::Fwd1Params p;
+  p.N = N;
+  p.BH = BH;
+  p.num_units = BH * ((N + attn::kBlockM - 1) / attn::kBlockM);
+  p.heads_per_group = heads_per_group(BH, N, D, MX ? 1 : 2, causal);
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.q_sf = static_cast<const uint8_t*>(q_sf);
+  p.k_sf = static_cast<const uint8_t*>(k_sf);
+  p.v_sf = static_cast<const uint8_t*>(v_sf);
+  p.timeout_cycles = kWaitLimitCycles;
+  const int sms = sm_count();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  const int grid = p.num_units < sms ? p.num_units : sms;
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  if (cudaGetLastError() != cudaSuccess) {
+    forget_smem(tag);
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
@@ -325,6 +367,14 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
     return ATTN_ERR_MISALIGNED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int BH = B * H;
+#ifndef ATTN_FWD_ONE_TILE
+#define ATTN_FWD_ONE_TILE 0
+#endif
+  if (ATTN_FWD_ONE_TILE) {
+    if (d == 128)
+      return launch_fwd1<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+    return launch_fwd1<64, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+  }
   if (d == 128)
     return launch_fwd<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
   return launch_fwd<64, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
@@ -359,6 +409,41 @@ attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const f
     return ATTN_ERR_MISALIGNED;
   return launch_fwd<128, true>(q8, k8, v8, o, lse, q_scale, k_scale, v_scale, B * H, N, scale, causal,
                                static_cast<cudaStream_t>(stream));
+}
+
+attn_status attn_quantize_mxfp8(const void* x, void* codes, void* sf, int B, int H, int N, int d, void* stream) {
+  if (x == nullptr || codes == nullptr || sf == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (d < 32 || d % 32 != 0 || d > 4096) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(sf)) return ATTN_ERR_MISALIGNED;
+  const long long nblk = static_cast<long long>(B) * H * N * (d / 32);
+  const int sms = sm_count();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  // 2048 threads per SM (8 CTAs of 256), fewer for small tensors: four lanes per block
+  const long long need = (nblk * 4 + attn::kMxQuantThreads - 1) / attn::kMxQuantThreads;
+  const long long cap = 8ll * sms;
+  const int grid = static_cast<int>(need < cap ? need : cap);
+  attn::mxfp8_quantize_sm100<<<grid, attn::kMxQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(codes), static_cast<uint8_t*>(sf), nblk);
+  if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  return ATTN_OK;
+}
+
+attn_status attn_fwd_mxfp8(const void* q8, const void* k8, const void* v8, const void* q_sf, const void* k_sf,
+                           const void* v_sf, void* o, float* lse, int B, int H, int N, int d, float scale,
+                           int causal, void* stream) {
+  if (q8 == nullptr || k8 == nullptr || v8 == nullptr || o == nullptr || q_sf == nullptr || k_sf == nullptr ||
+      v_sf == nullptr)
+    return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = resolve_scale(scale, d); s != ATTN_OK) return s;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(q_sf) || !aligned16(k_sf) ||
+      !aligned16(v_sf) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
+    return ATTN_ERR_MISALIGNED;
+  return launch_fwd1<128, true>(q8, k8, v8, o, lse, q_sf, k_sf, v_sf, B * H, N, scale, causal,
+                                static_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* scales, int B, int H, int N, int d,

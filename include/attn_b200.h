@@ -13,7 +13,8 @@
  *
  * Conventions shared by every entry point
  *   - Tensors are dense, contiguous, row-major [B, H, N, d] with d innermost;
- *     LSE is [B, H, N]; per-tile FP8 scales are [B, H, ceil(N/128)].
+ *     LSE is [B, H, N]; per-tile FP8 scales are [B, H, ceil(N/128)]; MXFP8
+ *     scale bytes are [B, H, N, d/32].
  *   - Every pointer argument is a DEVICE pointer owned by the caller, 16-byte
  *     aligned. The library never frees or retains caller memory.
  *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed as
@@ -115,13 +116,55 @@ ATTN_API attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8,
  *                a negative, infinite or NaN scale gives an undefined result.
  *   o   : [B, H, N, d] bf16 output.  lse: [B, H, N] fp32 or NULL.
  *   d   : 128 (else ATTN_ERR_UNSUPPORTED).
- * P is re-quantised on chip for the P V product (two E4M3 terms per value);
- * the error this adds is within the FP8 tolerance of the tests.
+ * S = Q K^T runs on the E4M3 tensor-core MMA; for P V the E4M3 V tile is
+ * widened on chip to f16 (exactly) and P is written as f16, with fp32
+ * accumulation; the error this adds is within the FP8 tolerance of the tests.
  */
 ATTN_API attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8,
                          const float* q_scale, const float* k_scale, const float* v_scale,
                          void* o, float* lse, int B, int H, int N, int d, float scale,
                          int causal, void* stream);
+
+/*
+ * attn_quantize_mxfp8 - MXFP8 quantisation of one tensor ("Efficient MoE
+ * training for biological foundation models", the low-precision paragraph:
+ * MXFP8, 8-bit values sharing one power-of-two scale per block of 32, the input
+ * format of Blackwell's block-scaled tensor-core products; the arithmetic below
+ * is the OCP Microscaling definition).
+ *   x     : [B, H, N, d] bf16 input, finite values.
+ *   codes : [B, H, N, d] output E4M3 codes (one byte each).
+ *   sf    : [B, H, N, d/32] output E8M0 scale bytes, one per 32 consecutive
+ *           values of a row (value 2^(byte - 127)).
+ *   d     : a multiple of 32, at most 4096 (else ATTN_ERR_UNSUPPORTED).
+ * Definition, per block: E = floor(log2(max |v|)) - 8 clamped to [-127, 127]
+ * (E = 0 for an all-zero block); byte = E + 127; code = E4M3 round-to-nearest-
+ * even, saturating to +-448, of v * 2^-E. Bit-exact with that definition.
+ */
+ATTN_API attn_status attn_quantize_mxfp8(const void* x, void* codes, void* sf, int B, int H, int N, int d,
+                                void* stream);
+
+/*
+ * attn_fwd_mxfp8 - attention forward on MXFP8 inputs (same page and paragraph as
+ * attn_quantize_mxfp8; what is computed is the attention of "Self-Attention,
+ * CUDA kernels and FlashAttention", section 1, eq. Attention, on the
+ * dequantised values decode(code) * 2^(byte - 127)).
+ *   q8, k8, v8       : [B, H, N, d] E4M3 codes.
+ *   q_sf, k_sf, v_sf : [B, H, N, d/32] E8M0 scale bytes (as attn_quantize_mxfp8
+ *                      writes them), 16-byte aligned.
+ *   o   : [B, H, N, d] bf16 output.  lse: [B, H, N] fp32 or NULL.
+ *   d   : 128 (else ATTN_ERR_UNSUPPORTED).
+ * S = Q K^T runs on the block-scaled MMA (tcgen05 kind::mxf8f6f4.block_scale:
+ * the scales are applied inside the tensor cores). V's blocks run along d, not
+ * along the keys P V contracts over, so V is widened on chip to f16 with its
+ * scales applied relative to the largest scale of its 32-column block over the
+ * keys a 128-row query tile sees: exact for every block within 22 binades of
+ * that largest scale (smaller blocks, below 2^-22 of the column's largest
+ * values, round in f16's subnormal range or flush to zero). P is written as
+ * f16; accumulation in fp32.
+ */
+ATTN_API attn_status attn_fwd_mxfp8(const void* q8, const void* k8, const void* v8, const void* q_sf,
+                           const void* k_sf, const void* v_sf, void* o, float* lse, int B, int H, int N,
+                           int d, float scale, int causal, void* stream);
 
 /*
  * attn_bwd - backward pass of attn_fwd (BF16) from the saved statistic LSE

@@ -61,3 +61,25 @@ def test_invariants_on_random_rows():
     _, sb2 = mx_quantize(y)
     changed = np.argwhere(sb2 != sb)
     assert all((r, b) == (10, 2) for r, b in changed)
+
+
+def test_ties_subnormals_and_exponent_clamps():
+    """Worked by hand. A block whose maximum is 256 has E = 0, so its other values
+    are encoded as they are: 1.0625 lies halfway between 1.0 (0x38) and 1.125
+    (0x39) and goes to the even mantissa, 1.0; 1.1875 lies halfway between 1.125
+    and 1.25 (0x3A) and goes to 1.25; 3 * 2^-9 is the subnormal code 3; 2^-10 is
+    halfway between 0 and the smallest subnormal 2^-9 and goes to 0; 3 * 2^-10 is
+    halfway between codes 1 and 2 and goes to 2. A block whose maximum is 2^-125
+    would need E = -133 and is clamped to E = -127 (byte 0), so 2^-125 is encoded
+    as 4.0 (0x48); a block whose maximum is 1.5 * 2^127 has E = 119 (byte 246)
+    and 384 (0x7C)."""
+    x = np.zeros((1, 96))
+    x[0, :6] = [256.0, 1.0625, 1.1875, 3 * 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -10]
+    x[0, 32] = 2.0 ** -125
+    x[0, 64] = 1.5 * 2.0 ** 127
+    codes, sb = mx_quantize(x)
+    assert sb.tolist() == [[127, 0, 246]]
+    assert codes[0, :6].tolist() == [0x78, 0x38, 0x3A, 0x03, 0x00, 0x02]
+    assert codes[0, 32] == 0x48 and codes[0, 64] == 0x7C
+    deq = mx_dequantize(codes, sb)
+    assert deq[0, 32] == 2.0 ** -125 and deq[0, 64] == 1.5 * 2.0 ** 127

@@ -306,6 +306,30 @@ def test_fp8_small_parity(cuda_lib, shape, causal):
     assert np.abs(lse - l_ref).max() <= TOL_LSE
 
 
+def test_fp8_every_code_through_pv_exact(cuda_lib):
+    """One key per head: P = 1, so O is the dequantised V itself. V holds every
+    finite E4M3 code (0x7F / 0xFF are the format's NaNs, never written by the
+    quantiser) and O must equal decode(code) * scale bit for bit (every such
+    value is a bf16 value): the on-chip widening of V is exact."""
+    from oracle.fp8 import e4m3_decode
+    dev = torch.device("cuda:0")
+    B, H, N, d = 1, 2, 1, 128
+    codes = np.arange(256, dtype=np.uint8)
+    codes[codes == 0x7F] = 0x00
+    codes[codes == 0xFF] = 0x80
+    v8 = torch.from_numpy(codes.reshape(B, H, N, d).copy()).to(dev)
+    zero8 = torch.zeros((B, H, N, d), dtype=torch.uint8, device=dev)
+    one = torch.ones((B, H, 1), dtype=torch.float32, device=dev)
+    vs = torch.tensor([1.0, 0.125], dtype=torch.float32, device=dev).view(B, H, 1)
+    o, lse = cuda_lib.forward_fp8(zero8, zero8, v8, one, one, vs)
+    torch.cuda.synchronize()
+    assert cuda_lib.attn_get_device_status(None) == cuda_lib.ATTN_OK
+    ref = e4m3_decode(codes).reshape(B, H, N, d) * np.array([1.0, 0.125]).reshape(B, H, 1, 1)
+    assert np.array_equal(ref, torch.from_numpy(ref).to(torch.bfloat16).double().numpy())
+    assert np.array_equal(o.double().cpu().numpy(), ref)
+    assert np.all(lse.cpu().numpy() == 0.0)
+
+
 def test_fp8_zero_scale_tiles(cuda_lib):
     """Tiles whose scale is 0 dequantise to zeros: a zero V tile contributes
     nothing and a zero K tile gives scores of exactly 0, with no NaN anywhere."""

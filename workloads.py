@@ -9,6 +9,9 @@ Workload shapes follow the pages:
     heads ("Self-Attention, CUDA kernels and FlashAttention", §1, patch grid and
     multi-head paragraph); head width 64.
   * LLM training and long-sequence shapes with head width 128 and causal masking.
+  * MXFP8 shape: the FP8 shape and outliers, quantised in 32-value blocks along d
+    ("Efficient MoE training for biological foundation models", the
+    low-precision paragraph).
   * FP8 shape: Q, K and V drawn with rare large outliers; Q and K are later
     multiplied by a random orthogonal matrix before block quantisation
     ("FlashAttention scaling, multi-GPU training and weight quantization", §1,
@@ -44,6 +47,7 @@ class Workload:
     d: int
     causal: bool
     fp8: bool = False
+    mx: bool = False              # MXFP8 inputs (32-value blocks, no rotation)
     outliers: tuple = ()          # subset of ("q", "k", "v")
     seed: int = 0
 
@@ -73,6 +77,10 @@ WORKLOADS = {
     # entries |O| reaches 20, where one bf16 step of the output is 0.125)
     "noncausal_8k_bf16": Workload("noncausal_8k_bf16", 2, 32, 8192, 128, False,
                                   outliers=("q", "k"), seed=1005),
+    # the FP8 workload's shape and outlier recipe, quantised to MXFP8 (one
+    # power-of-two scale per 32 values of a row; no rotation)
+    "mxfp8_8k": Workload("mxfp8_8k", 2, 32, 8192, 128, False, mx=True,
+                         outliers=("q", "k", "v"), seed=1007),
 }
 
 OUTLIER_FRACTION = 0.001
