@@ -31,9 +31,10 @@
 //    running byte-wise maximum of the V scale words of every key row it passes),
 //    so no value passes between the groups.
 //
-// CTA: 8 warps. warps 0-3 softmax (one thread per query row; warp w reads TMEM
-// lanes 32 w .. 32 w + 31), warp 4 TMA producer, warp 5 MMA issuer (owns TMEM),
-// warps 6-7 MXFP8 V conversion (idle for BF16).
+// CTA: warps 0-3 softmax (one thread per query row; warp w reads TMEM lanes
+// 32 w .. 32 w + 31), warp 4 TMA producer, warp 5 MMA issuer (owns TMEM); BF16:
+// 8 warps (6-7 idle); MXFP8: 12 warps, 6-9 the V conversion (one per SM
+// sub-partition), 10-11 idle, registers re-split per warpgroup.
 // TMEM (512 columns): S buffers [0, 128) and [128, 256) (P over their first 64
 // columns), O [256, 256 + D). MXFP8 scale factors: Q [384, 388), K of S buffer b
 // [388 + 4 b, 392 + 4 b), in the layout the block-scaled MMA reads for M = N =
@@ -82,9 +83,18 @@ struct Fwd1Cfg {
   static constexpr int P_CHUNKS = ATTN_P_CHUNKS;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
   static constexpr uint32_t POLY_MASK = ATTN_FWD1_POLY_MASK;
-  static constexpr int THREADS = 256;
+  // MXFP8: 12 warps, the V conversion spread over four warps (6-9), one on each
+  // SM sub-partition next to its softmax warp; warps 10-11 idle. Register split
+  // (launch: 65536 / 384 -> 168 per thread = 64512 in total): softmax warpgroup
+  // 248, the other two warpgroups 128: 128 * 248 + 256 * 128 = 64512.
+  static constexpr int THREADS = MX ? 384 : 256;
   static constexpr int PRODUCER_WARP = 4;
   static constexpr int MMA_WARP = 5;
+  static constexpr int CONV_WARPS = MX ? 4 : 0;
+  static constexpr int CONV_ITERS = MX ? 128 * 8 / (32 * CONV_WARPS) : 1;   // (row, 16-code unit) pairs per thread
+  static constexpr uint32_t REGS_SOFTMAX = 248;
+  static constexpr uint32_t REGS_OTHER = 128;
+  static_assert(!MX || 128 * REGS_SOFTMAX + 256 * REGS_OTHER <= 168 * THREADS, "register split");
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t O_COL0 = 256;
   static constexpr uint32_t SFA_COL = 384;
@@ -141,14 +151,29 @@ __device__ __forceinline__ void tmem_st4(uint32_t taddr, const uint32_t (&w)[4])
                : "memory");
 }
 
+// Read-only global loads issued exactly where they stand (volatile: the compiler
+// may neither sink them to their use nor reload them there), so that a load
+// issued a pipeline stage ahead keeps its latency hidden.
+__device__ __forceinline__ uint32_t ld_nc_u8(const uint8_t* ptr) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u8 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_nc_u32(const uint32_t* ptr) {
+  uint32_t v;
+  asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(ptr));
+  return v;
+}
+
 // Byte-wise maximum of two words of four scale bytes.
 __device__ __forceinline__ uint32_t max_u8x4(uint32_t a, uint32_t b) { return __vmaxu4(a, b); }
 
-// f16 bits of 2^x for x <= 15 (0 below f16's smallest subnormal 2^-24).
-__device__ __forceinline__ uint16_t f16_pow2_bits(int x) {
-  if (x >= -14) return static_cast<uint16_t>((x + 15) << 10);
-  if (x >= -24) return static_cast<uint16_t>(1u << (x + 24));
-  return 0;
+// f16 bits of 2^x for x <= 15 (0 below f16's smallest subnormal 2^-24), with
+// selects only (no branch: the lanes of a warp hold different x).
+__device__ __forceinline__ uint32_t f16_pow2_bits(int x) {
+  const uint32_t normal = static_cast<uint32_t>(max(x + 15, 0)) << 10;
+  const uint32_t sub = 1u << min(max(x + 24, 0), 31);
+  return x >= -14 ? normal : (x >= -24 ? sub : 0u);
 }
 
 // fp32 2^x for integer x in [-149, 127].
@@ -216,14 +241,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(q_empty, 1);
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(kv_full + i, 1);
-      mbar_init(kv_empty + i, (C::MX && (i & 1)) ? 2 : 1);   // MX V slots: the converter warps read them last
+      mbar_init(kv_empty + i, (C::MX && (i & 1)) ? C::CONV_WARPS : 1);   // MX V slots: the converter warps read them last
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(s_full + b, 1);
       for (int c = 0; c < C::P_CHUNKS; ++c) mbar_init(p_full + b * C::P_CHUNKS + c, 128);
       mbar_init(pv_done + b, 1);
       mbar_init(sfb_ready + b, 4);
-      mbar_init(vconv_full + b, 2);
+      mbar_init(vconv_full + b, C::CONV_WARPS > 0 ? C::CONV_WARPS : 1);
       mbar_init(vconv_empty + b, 1);
     }
     mbar_init(drain_bar, 1);
@@ -259,6 +284,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   if (warp == C::PRODUCER_WARP) {
     // ======================= TMA producer =======================
+    if constexpr (C::MX) regs_decrease<C::REGS_OTHER>();
     if (elect_one()) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
@@ -304,6 +330,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
   } else if (warp == C::MMA_WARP) {
     // ======================= MMA issuer =======================
+    if constexpr (C::MX) regs_decrease<C::REGS_OTHER>();
     // Per unit: S(0), S(1), then for each block j: P V(j) (chunk by chunk as P
     // arrives), then S(j + 2) into the buffer P(j) occupied. The tensor pipe runs
     // one thread's MMAs in issue order, so S(j + 2) overwrites P(j) only after
@@ -402,9 +429,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     __syncwarp();
   } else if (warp > C::MMA_WARP) {
     if constexpr (C::MX) {
+      regs_decrease<C::REGS_OTHER>();
+    }
+    if (C::MX && warp <= C::MMA_WARP + C::CONV_WARPS) {
       // ======================= MXFP8 V -> f16 with its block scales =======================
-      // Thread ct handles (key row, 16-code unit) pairs ct, ct + 64, ...: key rows
-      // ct / 8 + 8 i, unit un = ct % 8 (d = 16 un .. 16 un + 15, block un / 2).
+      // Thread ct (0 .. 32 CONV_WARPS - 1) handles (key row, 16-code unit) pairs
+      // ct, ct + 32 CONV_WARPS, ...: key rows ct / 8 + (4 CONV_WARPS) i, unit
+      // un = ct % 8 (d = 16 un .. 16 un + 15, block un / 2).
+      constexpr int ITERS = C::CONV_ITERS;
+      constexpr int ROW_STEP = 4 * C::CONV_WARPS;
       const int ct = (warp - C::MMA_WARP - 1) * 32 + lane;
       const int un = ct & 7, blk_d = un >> 1;
       uint32_t g = 0, vb = 0;
@@ -416,32 +449,32 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int kend = min(nkv * kBlockN, p.N);
         // scale bytes of this thread's 16 key rows, loaded one tile ahead (keys past
         // N: marked 0xFFFF, their codes are zero-filled and their factor is 0)
-        auto load_e = [&](int jt, uint32_t (&e)[16]) {
+        auto load_e = [&](int jt, uint32_t (&e)[ITERS]) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int key = jt * kBlockN + (ct >> 3) + 8 * i;
-            e[i] = key < p.N ? static_cast<uint32_t>(__ldg(p.v_sf + (head_row0 + key) * 4 + blk_d)) : 0xFFFFu;
+          for (int i = 0; i < ITERS; ++i) {
+            const int key = jt * kBlockN + (ct >> 3) + ROW_STEP * i;
+            e[i] = key < p.N ? ld_nc_u8(p.v_sf + (head_row0 + key) * 4 + blk_d) : 0xFFFFu;
           }
         };
-        uint32_t e_next[16];
+        uint32_t e_next[ITERS];
         load_e(0, e_next);
         const int sv = static_cast<int>((head_sf_max(p.v_sf, head_row0, kend, lane) >> (8 * blk_d)) & 0xFFu);
         for (int j = 0; j < nkv; ++j, ++vb) {
           const uint32_t vg = g + 2 * j + 1, vslot = vg % C::NSLOT, b = vb & 1;
-          uint32_t e_cur[16];
+          uint32_t e_cur[ITERS];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) e_cur[i] = e_next[i];
+          for (int i = 0; i < ITERS; ++i) e_cur[i] = e_next[i];
           if (j + 1 < nkv) load_e(j + 1, e_next);
           if (!(ok = wait_all(kv_full + vslot, (vg / C::NSLOT) & 1))) break;
           if (vb >= 2 && !(ok = wait_all(vconv_empty + b, ((vb >> 1) - 1) & 1))) break;
           const uint8_t* src = smem + C::SMEM_KV + vslot * C::TILE_BYTES;
           uint8_t* dst = smem + C::SMEM_VCONV + b * C::VCONV_BYTES;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int r = (ct >> 3) + 8 * i;
+          for (int i = 0; i < ITERS; ++i) {
+            const int r = (ct >> 3) + ROW_STEP * i;
             // f16 factor 2^(e - sv + 7)
-            const uint16_t sb = e_cur[i] != 0xFFFFu ? f16_pow2_bits(static_cast<int>(e_cur[i]) - sv + 7) : 0;
-            const uint32_t s2u = static_cast<uint32_t>(sb) * 0x10001u;
+            const uint32_t sb = e_cur[i] != 0xFFFFu ? f16_pow2_bits(static_cast<int>(e_cur[i]) - sv + 7) : 0u;
+            const uint32_t s2u = sb * 0x10001u;
             const __half2 s2 = *reinterpret_cast<const __half2*>(&s2u);
             const uint4 c16 = *reinterpret_cast<const uint4*>(src + r * 128 + ((un ^ (r & 7)) << 4));
             const uint32_t wds[4] = {c16.x, c16.y, c16.z, c16.w};
@@ -474,6 +507,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   } else {
     // ======================= softmax: one thread per query row =======================
+    if constexpr (C::MX) regs_increase<C::REGS_SOFTMAX>();
     const int r = warp * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t o_tm = tmem_base + lane_off + C::O_COL0;
@@ -484,7 +518,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         const int rr = row0 + 32 * h + lane;
-        wv[h] = rr < p.N ? __ldg(reinterpret_cast<const uint32_t*>(sf) + hrow0 + rr) : 0x7F7F7F7Fu;
+        wv[h] = rr < p.N ? ld_nc_u32(reinterpret_cast<const uint32_t*>(sf) + hrow0 + rr) : 0x7F7F7F7Fu;
       }
     };
     auto sf_store = [&](const uint8_t* sf, size_t hrow0, int row0, uint32_t col) {
@@ -546,7 +580,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int key = j * kBlockN + lane + 32 * i;
-            vw[i] = key < p.N ? __ldg(reinterpret_cast<const uint32_t*>(p.v_sf) + head_row0 + key) : 0u;
+            vw[i] = key < p.N ? ld_nc_u32(reinterpret_cast<const uint32_t*>(p.v_sf) + head_row0 + key) : 0u;
           }
           if (j + 2 < nkv)
             sf_load(p.k_sf, head_row0, (j + 2) * kBlockN, wa);
