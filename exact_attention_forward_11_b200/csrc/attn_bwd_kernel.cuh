@@ -62,7 +62,7 @@ struct BwdCfg {
   static constexpr int THREADS = 128 + 128 * SPLIT;
   static constexpr int COMPUTE_WARP0 = 4;
   static constexpr uint32_t TMEM_COLS = 512;
-  // dkdv shared memory: K, V, then per stage {Q, dO, lse2[128], D[128]}
+  // dkdv shared memory: K, V, then per stage {Q, dO, LSE[128], D[128]}
   static constexpr int DKDV_K = 0;
   static constexpr int DKDV_V = TILE_BYTES;
   static constexpr int DKDV_STAGE = 2 * TILE_BYTES;
@@ -286,14 +286,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           tma_load_3d(stage_do(s) + c * C::CHUNK_BYTES, &tm_do, q_full + s, c * 64, i * 128, bh, pol_q);
         }
       }
-      // the block's row statistics: LSE in log2 units (+inf past N, so P = 0 there) and D
+      // the block's row statistics LSE and D, copied asynchronously (zeros past N;
+      // the compute threads mask those queries): each lane's copies arrive on the
+      // stage's barrier when they land, so the producer never waits for them
       for (int t = lane; t < 128; t += 32) {
         const int q = i * 128 + t;
-        const size_t g = static_cast<size_t>(bh) * p.N + q;
-        stage_lse(s)[t] = q < p.N ? p.lse[g] * kLog2e : __int_as_float(0x7f800000);
-        stage_dd(s)[t] = q < p.N ? p.dd[g] : 0.f;
+        const bool in = q < p.N;
+        const size_t g = static_cast<size_t>(bh) * p.N + (in ? q : 0);
+        cp_async_4(stage_lse(s) + t, p.lse + g, in);
+        cp_async_4(stage_dd(s) + t, p.dd + g, in);
       }
-      mbar_arrive(q_full + s);
+      cp_async_arrive_noinc(q_full + s);
       __syncwarp();
     }
     if (!ok) {
@@ -382,17 +385,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           __syncwarp();
           if (lane == 0) mbar_arrive(s_read);
         }
-        // visible: key < N, and for the diagonal block of a causal launch, key <= query
+        // visible: key < N, query < N, and for the diagonal block of a causal
+        // launch, key <= query
         const int first_visible = (key >= p.N) ? 128 : ((p.causal && i == jb) ? r : 0);
+        const int end_visible = p.N - i * 128;            // queries past N read LSE = D = 0
 #pragma unroll
         for (int j4 = 0; j4 < NCOL / 4; ++j4) {
           const float4 l4 = lse2[j4];
-          const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+          const float lv[4] = {l4.x * kLog2e, l4.y * kLog2e, l4.z * kLog2e, l4.w * kLog2e};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int j = 4 * j4 + e;
             const float x = ex2_approx(fmaf(__uint_as_float(sr[j]), c, -lv[e]));
-            pr[j] = (col0 + j >= first_visible) ? x : 0.f;
+            pr[j] = (col0 + j >= first_visible && col0 + j < end_visible) ? x : 0.f;
           }
         }
         uint32_t pk[NCOL / 2];
