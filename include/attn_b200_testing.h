@@ -2,9 +2,12 @@
  * attn_b200_testing.h - testing hook of the attention library (not part of the
  * operation; the pages define no counterpart).
  *
- * attn_fwd_inject_timeout - attn_fwd for BF16, d = 128, with one failure
- * planted on purpose so that the bounded-wait path of the kernel can be run on
- * a GPU without faulting it: the TMA producer of the CTA that processes work
+ * attn_fwd_inject_timeout - attn_fwd for BF16, d = 128, always on the
+ * two-Q-tile schedule (attn_fwd itself runs launches with fewer two-tile units
+ * than SMs on the one-tile schedule, which gives bit-identical results), with
+ * one failure planted on purpose so that the bounded-wait path of the kernel
+ * can be run on a GPU without faulting it (a fault_unit at or past the number
+ * of units plants nothing): the TMA producer of the CTA that processes work
  * unit `fault_unit` never loads that unit's first K tile, so the mbarrier the
  * MMA warp waits on is never completed. Every pipeline wait of the launch
  * gives up after `wait_limit_cycles` SM cycles (instead of the 2^31 that

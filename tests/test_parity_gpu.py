@@ -394,3 +394,27 @@ def test_fp8_workload_parity(cuda_lib):
     lse = lse.cpu().numpy().reshape(w.B * w.H, w.N)[heads][:, rows]
     assert np.abs(o - o_ref).max() <= TOL_FP8
     assert np.abs(lse - l_ref).max() <= TOL_LSE
+
+
+def test_one_tile_and_two_tile_schedules_agree(cuda_lib):
+    """attn_fwd runs launches with fewer two-Q-tile units than SMs on the one-Q-tile
+    schedule (attn_fwd1_kernel.cuh); the testing hook attn_fwd_inject_timeout with
+    no tile withheld runs any shape on the two-tile schedule (attn_fwd_kernel.cuh).
+    Both take every row through the same operations in the same order, so O and LSE
+    agree bit for bit, and a head-sharded run gives the same bytes whichever
+    schedule each shard's size selects."""
+    dev = torch.device("cuda:0")
+    # (the hook takes d = 128 only)
+    for (B, H, N, d, causal) in [(2, 3, 300, 128, False), (2, 3, 300, 128, True), (1, 4, 257, 128, True),
+                                 (1, 2, 1000, 128, False), (1, 1, 129, 128, False)]:
+        q, k, v = (x.to(dev) for x in workloads.make_qkv(B, H, N, d, seed=N + d))
+        o1, l1 = cuda_lib.forward(q, k, v, causal=causal)
+        o2 = torch.empty_like(o1)
+        l2 = torch.empty_like(l1)
+        st = cuda_lib.attn_fwd_inject_timeout(q.data_ptr(), k.data_ptr(), v.data_ptr(), o2.data_ptr(), l2.data_ptr(),
+                                              B, H, N, d, 0.0, int(causal), 1 << 30, 1 << 31, None)
+        assert st == cuda_lib.ATTN_OK
+        torch.cuda.synchronize()
+        assert cuda_lib.attn_get_device_status(None) == cuda_lib.ATTN_OK
+        assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)), (B, H, N, d, causal)
+        assert torch.equal(l1.view(torch.int32), l2.view(torch.int32)), (B, H, N, d, causal)
