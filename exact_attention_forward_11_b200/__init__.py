@@ -3,7 +3,7 @@
 The entry points below have the names and arguments of include/attn_b200.h and
 only marshal arguments: every step of the computation runs in the CUDA kernels
 of libattn_b200.so. There is no CPU fallback; if the library is missing the
-calls raise. `forward`, `quantize_fp8`, `forward_fp8`, `quantize_mxfp8`, `forward_mxfp8`,
+calls raise. `forward`, `forward_from_host`, `quantize_fp8`, `forward_fp8`, `quantize_mxfp8`, `forward_mxfp8`,
 `backward` and `w4a16_matmul` are torch conveniences
 that allocate outputs with torch (PyTorch serves only for device memory and
 streams) and call the same entry points.
@@ -189,6 +189,88 @@ def forward(q, k, v, causal=False, scale=None, out=None, lse=None, with_lse=True
     _check(attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), _ptr(lse), B, H, N, d, sc,
                     int(bool(causal)), ATTN_BF16, sp), "attn_fwd")
     _check_device(check, sp, "attn_fwd")
+    return out, lse
+
+
+_HOST_STREAMS = {}
+
+
+def forward_from_host(q, k, v, causal=False, scale=None, out=None, lse=None, device=None, chunks=8):
+    """O, LSE of attention for HOST tensors: bf16 [B, H, N, d] in (pinned) CPU
+    memory in, O bf16 [B, H, N, d] and LSE fp32 [B, H, N] in (pinned) CPU memory
+    out, for callers whose inputs arrive on the host.
+
+    The B*H heads are cut into `chunks` contiguous groups (the heads are
+    independent). Three streams overlap the copies with the kernels: group c+1
+    is copied in while attn_fwd runs on group c (pointer offsets into the device
+    buffers) and group c-1 is copied out, so the two PCIe directions and the GPU
+    work at the same time. Returns once O and LSE are in host memory and the
+    device status word reads ATTN_OK (raises AttnError otherwise). The results
+    are the same bytes as forward() on the same inputs."""
+    import torch
+
+    from .sharded import head_range
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda or t.dim() != 4 or not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError(f"{name} must be a contiguous bf16 CPU tensor [B, H, N, d]")
+    B, H, N, d = q.shape
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v shapes differ")
+    BH = B * H
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16).pin_memory()
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    if out.is_cuda or tuple(out.shape) != (B, H, N, d) or out.dtype != torch.bfloat16 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 CPU tensor [B, H, N, d]")
+    if lse.is_cuda or tuple(lse.shape) != (B, H, N) or lse.dtype != torch.float32 or not lse.is_contiguous():
+        raise ValueError("lse must be a contiguous fp32 CPU tensor [B, H, N]")
+    chunks = max(1, min(int(chunks), BH))
+    key = dev.index
+    if key not in _HOST_STREAMS:
+        _HOST_STREAMS[key] = tuple(torch.cuda.Stream(dev) for _ in range(3))
+    s_in, s_run, s_out = _HOST_STREAMS[key]
+    flat = [t.view(BH, N, d) for t in (q, k, v)]
+    o_flat, l_flat = out.view(BH, N, d), lse.view(BH, N)
+    dq, dk, dv, do = (torch.empty((BH, N, d), dtype=torch.bfloat16, device=dev) for _ in range(4))
+    # one LSE buffer per group: an offset of h0 * N floats into a shared one is
+    # 16-byte aligned only when h0 * N is a multiple of 4
+    dls = [torch.empty((head_range(BH, chunks, c)[1], N), dtype=torch.float32, device=dev) for c in range(chunks)]
+    # the device buffers are allocated on the current stream; the three streams
+    # start after it
+    start = torch.cuda.Event()
+    start.record(torch.cuda.current_stream(dev))
+    for st in (s_in, s_run, s_out):
+        st.wait_event(start)
+    sc = 0.0 if scale is None else float(scale)
+    elem = 2 * N * d
+    for c in range(chunks):
+        h0, cnt = head_range(BH, chunks, c)
+        if cnt == 0:
+            continue
+        sl = slice(h0, h0 + cnt)
+        with torch.cuda.stream(s_in):
+            for dst, src in zip((dq, dk, dv), flat):
+                dst[sl].copy_(src[sl], non_blocking=True)
+            ready = torch.cuda.Event()
+            ready.record(s_in)
+        s_run.wait_event(ready)
+        off = h0 * elem
+        _check(attn_fwd(dq.data_ptr() + off, dk.data_ptr() + off, dv.data_ptr() + off, do.data_ptr() + off,
+                        dls[c].data_ptr(), 1, cnt, N, d, sc, int(bool(causal)), ATTN_BF16,
+                        s_run.cuda_stream), "attn_fwd")
+        done = torch.cuda.Event()
+        done.record(s_run)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            o_flat[sl].copy_(do[sl], non_blocking=True)
+            l_flat[sl].copy_(dls[c], non_blocking=True)
+    # every copy and launch above has finished once the copy-out stream has (it
+    # waited on each group's kernel, which waited on that group's copies in), so
+    # the device buffers can go back to the allocator when this returns
+    s_out.synchronize()
+    _check(attn_get_device_status(s_run.cuda_stream), "forward_from_host (device status)")
     return out, lse
 
 

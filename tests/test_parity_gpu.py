@@ -418,3 +418,19 @@ def test_one_tile_and_two_tile_schedules_agree(cuda_lib):
         assert cuda_lib.attn_get_device_status(None) == cuda_lib.ATTN_OK
         assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)), (B, H, N, d, causal)
         assert torch.equal(l1.view(torch.int32), l2.view(torch.int32)), (B, H, N, d, causal)
+
+
+def test_forward_from_host_matches_forward(cuda_lib):
+    """The host-to-host entry (inputs copied in and outputs copied out by head
+    groups on three streams) returns the same bytes as forward() on device
+    copies, for any number of groups (including more groups than heads) and for
+    N that is not a multiple of 4 (per-group LSE buffers)."""
+    dev = torch.device("cuda:0")
+    for (B, H, N, d, causal), chunks in [((2, 3, 300, 128, True), 4), ((1, 5, 257, 64, False), 1),
+                                          ((1, 2, 129, 128, False), 7), ((3, 4, 1000, 128, True), 3)]:
+        q, k, v = (x.pin_memory() for x in workloads.make_qkv(B, H, N, d, seed=N + 3 * d))
+        o_h, l_h = cuda_lib.forward_from_host(q, k, v, causal=causal, chunks=chunks)
+        o_d, l_d = cuda_lib.forward(q.to(dev), k.to(dev), v.to(dev), causal=causal)
+        torch.cuda.synchronize()
+        assert torch.equal(o_h.view(torch.int16), o_d.cpu().view(torch.int16)), (B, H, N, d, causal, chunks)
+        assert torch.equal(l_h.view(torch.int32), l_d.cpu().view(torch.int32)), (B, H, N, d, causal, chunks)
