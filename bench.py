@@ -294,9 +294,13 @@ class Step:
             self.codes = [torch.empty((w.B, w.H, w.N, w.d), device=dev, dtype=torch.uint8) for _ in range(3)]
             self.sfs = [torch.empty((w.B, w.H, w.N, w.d // 32), device=dev, dtype=torch.uint8) for _ in range(3)]
         self.launches = 4 if (w.fp8 or w.mx) else 1
-        self.attn_kernel = "attn_fwd1_sm100" if w.mx else "attn_fwd_sm100"
+        # attn_fwd runs launches with fewer two-Q-tile units than SMs on the
+        # one-tile kernel (attn_fwd1_sm100), the rest on the two-tile kernel
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        one_tile = w.B * w.H * ((w.N + 255) // 256) < sms
+        self.attn_kernel = "attn_fwd1_sm100" if (w.mx or (one_tile and not w.fp8)) else "attn_fwd_sm100"
         self.kernels = (["fp8_rotate_quantize", "fp8_quantize", "attn_fwd_sm100"] if w.fp8
-                        else ["mxfp8_quantize", "attn_fwd1_sm100"] if w.mx else ["attn_fwd_sm100"])
+                        else ["mxfp8_quantize", "attn_fwd1_sm100"] if w.mx else [self.attn_kernel])
 
     def run_device(self, stream, mark=None):
         """Launches one step on `stream`; mark(kernel name), if given, is called
@@ -324,7 +328,7 @@ class Step:
                               w.B, w.H, w.N, w.d, w.scale, int(w.causal), lib.ATTN_BF16, s)
             if st:
                 raise lib.AttnError(st, "attn_fwd")
-            mark("attn_fwd_sm100")
+            mark(self.attn_kernel)
             return
         for src, rot, c8, sc in zip((self.q, self.k, self.v), (self.rot, self.rot, None), self.codes, self.scales):
             st = lib.attn_quantize_fp8(src.data_ptr(), None if rot is None else rot.data_ptr(), c8.data_ptr(),
