@@ -33,6 +33,7 @@ SIGNATURES = {
     "attn_fwd_mxfp8": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "attn_get_device_status": (_I, [_P]),
     "attn_fwd_inject_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, ctypes.c_ulonglong, _P]),
+    "attn_fwd_one_tile_inject_timeout": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I, ctypes.c_ulonglong, _P]),
     "attn_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _I, _F, _I, _P]),
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
@@ -110,6 +111,13 @@ def attn_fwd_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_un
     """Testing hook (include/attn_b200_testing.h): attn_fwd with one K tile withheld."""
     return load().attn_fwd_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit,
                                           wait_limit_cycles, stream)
+
+
+def attn_fwd_one_tile_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit, wait_limit_cycles,
+                                     stream):
+    """Testing hook (include/attn_b200_testing.h): the one-Q-tile schedule with one K tile withheld."""
+    return load().attn_fwd_one_tile_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit,
+                                                   wait_limit_cycles, stream)
 
 
 def attn_get_device_status(stream):

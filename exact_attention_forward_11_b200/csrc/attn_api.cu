@@ -241,7 +241,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
 template <int D, bool MX>
 attn_status launch_fwd1(const void* q, const void* k, const void* v, void* o, float* lse, const void* q_sf,
                         const void* k_sf, const void* v_sf, int BH, int N, float scale, int causal,
-                        cudaStream_t stream) {
+                        cudaStream_t stream, int fault_unit = -1, uint64_t wait_limit = kWaitLimitCycles) {
   using C = attn::Fwd1Cfg<D, MX>;
   auto kern = attn::attn_fwd1_sm100<C>;
   const int tag = MX ? 12 : (D == 128 ? 10 : 11);
@@ -262,7 +262,8 @@ attn_status launch_fwd1(const void* q, const void* k, const void* v, void* o, fl
   p.q_sf = static_cast<const uint8_t*>(q_sf);
   p.k_sf = static_cast<const uint8_t*>(k_sf);
   p.v_sf = static_cast<const uint8_t*>(v_sf);
-  p.timeout_cycles = kWaitLimitCycles;
+  p.timeout_cycles = wait_limit;
+  p.fault_unit = fault_unit;
   const int sms = sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
   const int grid = p.num_units < sms ? p.num_units : sms;
@@ -400,6 +401,21 @@ attn_status attn_fwd_inject_timeout(const void* q, const void* k, const void* v,
     return ATTN_ERR_MISALIGNED;
   return launch_fwd<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, B * H, N, scale, causal,
                                 static_cast<cudaStream_t>(stream), fault_unit, wait_limit_cycles);
+}
+
+attn_status attn_fwd_one_tile_inject_timeout(const void* q, const void* k, const void* v, void* o, float* lse,
+                                             int B, int H, int N, int d, float scale, int causal, int fault_unit,
+                                             unsigned long long wait_limit_cycles, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
+  if (attn_status s = resolve_scale(scale, d); s != ATTN_OK) return s;
+  if (attn_status s = check_shape(B, H, N); s != ATTN_OK) return s;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (fault_unit < 0 || wait_limit_cycles < 1024) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
+    return ATTN_ERR_MISALIGNED;
+  return launch_fwd1<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, B * H, N, scale, causal,
+                                 static_cast<cudaStream_t>(stream), fault_unit, wait_limit_cycles);
 }
 
 attn_status attn_fwd_fp8(const void* q8, const void* k8, const void* v8, const float* q_scale, const float* k_scale,

@@ -123,6 +123,7 @@ struct Fwd1Params {
   const uint8_t* k_sf;
   const uint8_t* v_sf;
   uint64_t timeout_cycles;   // per pipeline wait, in SM cycles
+  int fault_unit;            // testing only: the producer withholds this unit's first K tile (-1: none)
 };
 
 // Instruction descriptor of the block-scaled E4M3 x E4M3 MMA with fp32
@@ -308,6 +309,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       __syncwarp();
       ++units;
       for (int i = 0; i < 2 * w.nkv[0]; ++i, ++g) {
+        // testing hook: a tile that is never loaded leaves its full barrier
+        // incomplete, so the MMA warp's bounded wait runs out
+        if (i == 0 && u == p.fault_unit) continue;
         const uint32_t slot = g % C::NSLOT;
         if (g >= C::NSLOT && !(ok = wait_all(kv_empty + slot, ((g / C::NSLOT) - 1) & 1))) break;
         const CUtensorMap* tm = (i & 1) ? &tm_v : &tm_k;

@@ -38,6 +38,18 @@ ATTN_API attn_status attn_fwd_inject_timeout(const void* q, const void* k, const
                                              int B, int H, int N, int d, float scale, int causal, int fault_unit,
                                              unsigned long long wait_limit_cycles, void* stream);
 
+/*
+ * attn_fwd_one_tile_inject_timeout - the same hook on the one-Q-tile schedule
+ * (the kernel attn_fwd runs for launches with few units, and the one
+ * attn_fwd_mxfp8 runs): work unit u covers one head and ONE 128-row Q tile
+ * (u < B*H*ceil(N/128)), numbered as for the two-tile schedule with one tile per
+ * pair. Arguments, limits and results as for attn_fwd_inject_timeout.
+ */
+ATTN_API attn_status attn_fwd_one_tile_inject_timeout(const void* q, const void* k, const void* v, void* o,
+                                                      float* lse, int B, int H, int N, int d, float scale,
+                                                      int causal, int fault_unit,
+                                                      unsigned long long wait_limit_cycles, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -70,3 +70,42 @@ def test_inject_timeout_validates_arguments(cuda_lib):
     lib = cuda_lib
     bad = lib.attn_fwd_inject_timeout(0, 0, 0, 0, 0, 1, 1, 128, 128, 0.0, 0, 0, WAIT_LIMIT, None)
     assert bad == lib.ATTN_ERR_INVALID_ARG
+
+
+def test_one_tile_starved_unit_times_out_and_context_survives(cuda_lib):
+    """The same planted failure on the one-Q-tile schedule (the kernel behind
+    small attn_fwd launches and attn_fwd_mxfp8)."""
+    lib = cuda_lib
+    dev = torch.device("cuda:0")
+    B, H, N, d = 1, 4, 1024, 128          # 4 heads x 8 Q tiles = 32 units, one per CTA
+    q, k, v = _inputs(B, H, N, d, seed=2025)
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    o = torch.full((B, H, N, d), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+
+    fault_unit = 5                        # unit u -> tile 7 - u // 4 of head u % 4: head 1, rows 768..895
+    t0 = time.time()
+    st = lib.attn_fwd_one_tile_inject_timeout(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), o.data_ptr(),
+                                              lse.data_ptr(), B, H, N, d, 0.0, 0, fault_unit, WAIT_LIMIT, None)
+    assert st == lib.ATTN_OK, lib.attn_status_string(st)
+    assert lib.attn_get_device_status(None) == lib.ATTN_ERR_TIMEOUT
+    assert time.time() - t0 < 30.0
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+
+    o_h = o.float().cpu().numpy()
+    lse_h = lse.cpu().numpy()
+    scale = 1.0 / np.sqrt(d)
+    rows = np.array([0, 131, 517, 767, 896, 1023])
+    o_ref, lse_ref = attention_fp64(q.double().numpy(), k.double().numpy(), v.double().numpy(), scale, False,
+                                    rows=rows)
+    for h in range(H):                    # every tile but the starved one is exact, head 1 included
+        assert np.abs(o_h[0, h, rows] - o_ref[0, h]).max() <= 2e-2
+        assert np.abs(lse_h[0, h, rows] - lse_ref[0, h]).max() <= 1e-3
+
+    lib.forward(qd, kd, vd, causal=False, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+    o_ref, _ = attention_fp64(q.double().numpy(), k.double().numpy(), v.double().numpy(), scale, False,
+                              rows=np.arange(768, 896))
+    assert np.abs(o.float().cpu().numpy()[0, 1, 768:896] - o_ref[0, 1]).max() <= 2e-2
