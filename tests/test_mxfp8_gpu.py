@@ -278,3 +278,22 @@ def test_mx_every_code_through_pv_exact(cuda_lib):
     assert np.array_equal(o.double().cpu().numpy(), ref)
     assert np.all(lse.cpu().numpy() == 0.0)
     assert e4m3_decode(np.array([0x7E], dtype=np.uint8))[0] == 448.0
+
+
+def test_mx_long_causal_sampled(cuda_lib):
+    """A long causal launch (N = 16384: units of 1 to 128 key blocks, heaviest
+    first) on sampled rows, including the first and last rows of Q tiles."""
+    B, H, N, d = 1, 2, 16384, 128
+    q, k, v = workloads.make_qkv(B, H, N, d, seed=55, outliers=("q", "k"))
+    (q8, qs), (k8, ks), (v8, vs) = (gpu_quant(cuda_lib, x) for x in (q, k, v))
+    o, lse = cuda_lib.forward_mxfp8(q8, k8, v8, qs, ks, vs, causal=True)
+    torch.cuda.synchronize()
+    assert cuda_lib.attn_get_device_status(None) == cuda_lib.ATTN_OK
+    rows = sorted(set([0, 1, 127, 128, 4095, 8191, 8192, 16383] + workloads.sample_rows(N, 40, 9)))
+    o_ref, l_ref = reference(q, k, v, 1 / math.sqrt(d), True, rows=rows)
+    o_g = o.float().cpu().numpy()[:, :, rows]
+    l_g = lse.cpu().numpy()[:, :, rows]
+    err = np.abs(o_g - o_ref)
+    assert err.max() <= TOL_MAX, err.max()
+    assert err.mean() <= TOL_MEAN, err.mean()
+    assert np.abs(l_g - l_ref).max() <= TOL_LSE
