@@ -15,9 +15,13 @@ import math
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
+RELEASE_LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
+# the debug build (device-side index checks, ATTN_ERR_BOUNDS): ATTN_B200_DEBUG=1
+DEBUG_LIB_PATH = os.path.join(_HERE, "libattn_b200_debug.so")
+LIB_PATH = DEBUG_LIB_PATH if os.environ.get("ATTN_B200_DEBUG", "0") not in ("", "0") else RELEASE_LIB_PATH
 
-ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT = range(6)
+(ATTN_OK, ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED, ATTN_ERR_MISALIGNED, ATTN_ERR_CUDA, ATTN_ERR_TIMEOUT,
+ ATTN_ERR_BOUNDS) = range(7)
 ATTN_BF16 = 0
 TILE = 128
 
@@ -38,6 +42,9 @@ SIGNATURES = {
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "w4a16_gemm": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "attn_fwd_debug_row_limit": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, ctypes.c_longlong, _P]),
+    "attn_debug_build": (_I, []),
+    "attn_debug_last_failure": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_longlong), _P]),
     "attn_status_string": (ctypes.c_char_p, [_I]),
     "attn_abi_version": (_I, []),
 }
@@ -50,7 +57,8 @@ class AttnError(RuntimeError):
 
 
 def load():
-    """Load libattn_b200.so (built by exact_attention_forward_11_b200.build)."""
+    """Load the library at LIB_PATH: libattn_b200.so, or with ATTN_B200_DEBUG=1 its
+    debug build libattn_b200_debug.so (both built by exact_attention_forward_11_b200.build)."""
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
@@ -118,6 +126,35 @@ def attn_fwd_one_tile_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal,
     """Testing hook (include/attn_b200_testing.h): the one-Q-tile schedule with one K tile withheld."""
     return load().attn_fwd_one_tile_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit,
                                                    wait_limit_cycles, stream)
+
+
+def attn_fwd_debug_row_limit(q, k, v, o, lse, B, H, N, d, scale, causal, row_limit, stream):
+    """Testing hook of the debug build (include/attn_b200_testing.h): attn_fwd told
+    that O / LSE hold only `row_limit` rows."""
+    return load().attn_fwd_debug_row_limit(q, k, v, o, lse, B, H, N, d, scale, causal, row_limit, stream)
+
+
+def attn_debug_build():
+    return load().attn_debug_build()
+
+
+def attn_debug_last_failure(stream):
+    """(site, index) of the first debug check that failed since the last call; site 0: none."""
+    site, index = ctypes.c_int(0), ctypes.c_longlong(0)
+    st = load().attn_debug_last_failure(ctypes.byref(site), ctypes.byref(index), stream)
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_debug_last_failure")
+    return site.value, index.value
+
+
+def use_library(path):
+    """Switch the binding to another build of the library (e.g. DEBUG_LIB_PATH);
+    later calls go to it. Returns the previous path."""
+    global _lib, LIB_PATH
+    prev = LIB_PATH
+    LIB_PATH = path
+    _lib = None
+    return prev
 
 
 def attn_get_device_status(stream):

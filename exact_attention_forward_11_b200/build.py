@@ -1,6 +1,8 @@
-"""Builds the C-ABI shared library (libattn_b200.so) in-tree with nvcc for sm_100a.
+"""Builds the C-ABI shared library (libattn_b200.so) in-tree with nvcc for sm_100a,
+and its debug build (libattn_b200_debug.so: the same sources with -DATTN_DEBUG,
+device-side index checks that record ATTN_ERR_BOUNDS and skip the access).
 
-    python -m exact_attention_forward_11_b200.build
+    python -m exact_attention_forward_11_b200.build [--force] [--debug]
 """
 from __future__ import annotations
 
@@ -14,6 +16,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libattn_b200.so")
+LIB_DEBUG = os.path.join(HERE, "libattn_b200_debug.so")
 
 SOURCES = ["attn_api.cu"]
 HEADERS = ["sm100.cuh", "status.cuh", "attn_fwd_kernel.cuh", "attn_fwd1_kernel.cuh", "mxfp8_quant_kernel.cuh", "attn_bwd_kernel.cuh", "fp8_prep_kernel.cuh", "w4a16_kernel.cuh"]
@@ -31,26 +34,27 @@ def _nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, h) for h in os.listdir(INCLUDE)] + [__file__]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp"
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I" + INCLUDE, "-I" + CSRC, "-o", tmp,
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + ".tmp"
+    cmd = [_nvcc(), *NVCC_FLAGS, *(["-DATTN_DEBUG"] if debug else []), "-I" + INCLUDE, "-I" + CSRC, "-o", tmp,
            *[os.path.join(CSRC, s) for s in SOURCES]]
     if verbose:
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

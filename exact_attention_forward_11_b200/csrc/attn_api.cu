@@ -199,7 +199,8 @@ int heads_per_group(int BH, int N, int D, int elem, int causal) {
 template <int D, bool FP8>
 attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const float* qs,
                        const float* ks, const float* vs, int BH, int N, float scale, int causal,
-                       cudaStream_t stream, int fault_unit = -1, uint64_t wait_limit = kWaitLimitCycles) {
+                       cudaStream_t stream, int fault_unit = -1, uint64_t wait_limit = kWaitLimitCycles,
+                       long long out_rows = -1) {
   using C = attn::FwdCfg<D, FP8>;
   auto kern = attn::attn_fwd_sm100<C>;
   CUtensorMap tq, tk, tv;
@@ -223,6 +224,7 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
   p.v_scale = vs;
   p.timeout_cycles = wait_limit;
   p.fault_unit = fault_unit;
+  p.out_rows = static_cast<uint32_t>(out_rows < 0 ? static_cast<long long>(BH) * N : out_rows);
   // persistent grid: one CTA per SM (shared memory and TMEM allow one), each
   // walking the units blockIdx.x, blockIdx.x + gridDim.x, ...
   const int sms = sm_count();
@@ -241,7 +243,8 @@ attn_status launch_fwd(const void* q, const void* k, const void* v, void* o, flo
 template <int D, bool MX>
 attn_status launch_fwd1(const void* q, const void* k, const void* v, void* o, float* lse, const void* q_sf,
                         const void* k_sf, const void* v_sf, int BH, int N, float scale, int causal,
-                        cudaStream_t stream, int fault_unit = -1, uint64_t wait_limit = kWaitLimitCycles) {
+                        cudaStream_t stream, int fault_unit = -1, uint64_t wait_limit = kWaitLimitCycles,
+                        long long out_rows = -1) {
   using C = attn::Fwd1Cfg<D, MX>;
   auto kern = attn::attn_fwd1_sm100<C>;
   const int tag = MX ? 12 : (D == 128 ? 10 : 11);
@@ -264,6 +267,7 @@ attn_status launch_fwd1(const void* q, const void* k, const void* v, void* o, fl
   p.v_sf = static_cast<const uint8_t*>(v_sf);
   p.timeout_cycles = wait_limit;
   p.fault_unit = fault_unit;
+  p.out_rows = static_cast<uint32_t>(out_rows < 0 ? static_cast<long long>(BH) * N : out_rows);
   const int sms = sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
   const int grid = p.num_units < sms ? p.num_units : sms;
@@ -352,12 +356,19 @@ const char* attn_status_string(int status) {
     case ATTN_ERR_MISALIGNED: return "ATTN_ERR_MISALIGNED";
     case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
     case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    case ATTN_ERR_BOUNDS: return "ATTN_ERR_BOUNDS";
     default: return "ATTN_UNKNOWN_STATUS";
   }
 }
 
-attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
-                     float scale, int causal, attn_dtype dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// attn_fwd with the rows of O / LSE the kernels may write (-1: all B*H*N;
+// fewer only through the debug-build hook).
+attn_status fwd_bf16(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                     float scale, int causal, attn_dtype dtype, void* stream, long long out_rows) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return ATTN_ERR_INVALID_ARG;
   if (attn_status s = resolve_scale(scale, d); s != ATTN_OK) return s;
@@ -378,14 +389,56 @@ attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float
   const int sms = sm_count();
   if (sms <= 0) return ATTN_ERR_CUDA;
   const long long pair_units = static_cast<long long>(BH) * ((N + 2 * attn::kBlockM - 1) / (2 * attn::kBlockM));
+  const uint64_t wl = kWaitLimitCycles;
   if (ATTN_FWD_ONE_TILE || pair_units < sms) {
     if (d == 128)
-      return launch_fwd1<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
-    return launch_fwd1<64, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+      return launch_fwd1<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st, -1, wl,
+                                     out_rows);
+    return launch_fwd1<64, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st, -1, wl,
+                                  out_rows);
   }
   if (d == 128)
-    return launch_fwd<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
-  return launch_fwd<64, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st);
+    return launch_fwd<128, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st, -1, wl,
+                                  out_rows);
+  return launch_fwd<64, false>(q, k, v, o, lse, nullptr, nullptr, nullptr, BH, N, scale, causal, st, -1, wl,
+                               out_rows);
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int N, int d,
+                     float scale, int causal, attn_dtype dtype, void* stream) {
+  return fwd_bf16(q, k, v, o, lse, B, H, N, d, scale, causal, dtype, stream, -1);
+}
+
+attn_status attn_fwd_debug_row_limit(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                                     int N, int d, float scale, int causal, long long row_limit, void* stream) {
+  if (!attn::kDebugChecks) return ATTN_ERR_UNSUPPORTED;
+  if (B < 1 || H < 1 || N < 1 || row_limit < 0 || row_limit > static_cast<long long>(B) * H * N)
+    return ATTN_ERR_INVALID_ARG;
+  return fwd_bf16(q, k, v, o, lse, B, H, N, d, scale, causal, ATTN_BF16, stream, row_limit);
+}
+
+int attn_debug_build(void) { return attn::kDebugChecks ? 1 : 0; }
+
+attn_status attn_debug_last_failure(int* site, long long* index, void* stream) {
+  if (site == nullptr || index == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_CUDA;
+  uint32_t s = 0;
+  unsigned long long i = 0;
+  if (cudaMemcpyFromSymbol(&s, attn::g_debug_site, sizeof(s)) != cudaSuccess ||
+      cudaMemcpyFromSymbol(&i, attn::g_debug_index, sizeof(i)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  *site = static_cast<int>(s);
+  *index = static_cast<long long>(i);
+  const uint32_t zs = 0;
+  const unsigned long long zi = 0;
+  if (cudaMemcpyToSymbol(attn::g_debug_site, &zs, sizeof(zs)) != cudaSuccess ||
+      cudaMemcpyToSymbol(attn::g_debug_index, &zi, sizeof(zi)) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  return ATTN_OK;
 }
 
 attn_status attn_fwd_inject_timeout(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -598,7 +651,7 @@ attn_status attn_get_device_status(void* stream) {
   if (v == 0) return ATTN_OK;
   const uint32_t zero = 0;
   if (cudaMemcpyToSymbol(attn::g_status, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
-  return ATTN_ERR_TIMEOUT;
+  return (v & attn::kStatusBounds) ? ATTN_ERR_BOUNDS : ATTN_ERR_TIMEOUT;
 }
 
 }  // extern "C"

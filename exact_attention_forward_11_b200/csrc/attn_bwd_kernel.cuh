@@ -291,8 +291,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       // stage's barrier when they land, so the producer never waits for them
       for (int t = lane; t < 128; t += 32) {
         const int q = i * 128 + t;
-        const bool in = q < p.N;
-        const size_t g = static_cast<size_t>(bh) * p.N + (in ? q : 0);
+        const size_t gq = static_cast<size_t>(bh) * p.N + q;
+        const bool in = q < p.N && dbg_ok(gq < static_cast<size_t>(p.BH) * p.N, kSiteBwdStats, gq);
+        const size_t g = in ? gq : static_cast<size_t>(0);
         cp_async_4(stage_lse(s) + t, p.lse + g, in);
         cp_async_4(stage_dd(s) + t, p.dd + g, in);
       }
@@ -453,8 +454,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (ok) ok = wait_all(done, 0);
     if (ok) {
       tc_fence_after();
-      const bool in_range = key < p.N;
-      const size_t row = static_cast<size_t>(bh) * p.N + (in_range ? key : 0);
+      const size_t krow = static_cast<size_t>(bh) * p.N + key;
+      const bool in_range = key < p.N && dbg_ok(krow < static_cast<size_t>(p.BH) * p.N, kSiteBwdDkDv, krow);
+      const size_t row = in_range ? krow : static_cast<size_t>(0);
       if (C::SPLIT == 1 || h == 0)
         store_row_bf16<C::D>(tmem_base + lane_off + C::T_DV, 1.f, p.dv + row * C::D, in_range);
       if (C::SPLIT == 1 || h == 1)
@@ -627,9 +629,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int qrow = ib * 128 + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float c = p.scale_log2;
-    const size_t g = static_cast<size_t>(bh) * p.N + (qrow < p.N ? qrow : 0);
-    const float l2 = qrow < p.N ? p.lse[g] * kLog2e : __int_as_float(0x7f800000);
-    const float dd = qrow < p.N ? p.dd[g] : 0.f;
+    const size_t gq = static_cast<size_t>(bh) * p.N + qrow;
+    const bool q_in = qrow < p.N && dbg_ok(gq < static_cast<size_t>(p.BH) * p.N, kSiteBwdDq, gq);
+    const size_t g = q_in ? gq : static_cast<size_t>(0);
+    const float l2 = q_in ? p.lse[g] * kLog2e : __int_as_float(0x7f800000);
+    const float dd = q_in ? p.dd[g] : 0.f;
     for (int j = 0; j < n; ++j) {
       const uint32_t t_s = tmem_base + lane_off + C::T_S + 128 * (j & 1);
       if (!(ok = wait_all(s_full + (j & 1), (j >> 1) & 1))) break;
@@ -683,7 +687,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     if (ok) ok = wait_all(done, 0);
     if (ok) {
       tc_fence_after();
-      const bool in_range = qrow < p.N;
+      const bool in_range = q_in;
       // the two column halves of a row store the two halves of its dQ
       constexpr int DC = C::D / C::SPLIT;
       store_row_bf16<DC>(tmem_base + lane_off + C::T_DQ + DC * h, p.scale, p.dq + g * C::D + DC * h, in_range);

@@ -124,7 +124,13 @@ struct Fwd1Params {
   const uint8_t* v_sf;
   uint64_t timeout_cycles;   // per pipeline wait, in SM cycles
   int fault_unit;            // testing only: the producer withholds this unit's first K tile (-1: none)
+  uint32_t out_rows;         // rows of O and LSE the kernel may write (BH * N); checked in debug builds
 };
+
+// (debug builds) a scale-byte row index inside the [BH * N] arrays
+__device__ __forceinline__ bool sf_row_ok(const Fwd1Params& p, size_t r) {
+  return dbg_ok(r < static_cast<size_t>(p.BH) * p.N, kSiteFwd1ScaleLoad, r);
+}
 
 // Instruction descriptor of the block-scaled E4M3 x E4M3 MMA with fp32
 // accumulation and UE8M0 scales, both operands K-major; sf_id picks the scale
@@ -302,7 +308,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (units > 0 && !(ok = wait_all(q_empty, (units - 1) & 1))) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(q_full, C::TILE_BYTES);
-        for (int c = 0; c < C::CHUNKS; ++c)
+        // (debug) a unit outside the launch's heads or Q tiles loads nothing
+        const bool unit_ok = dbg_ok(w.bh < p.BH && w.qpair * kBlockM < p.N, kSiteTmaCoord, static_cast<unsigned>(u));
+        for (int c = 0; c < C::CHUNKS && unit_ok; ++c)
           tma_load_3d(smem + C::SMEM_Q + c * C::CHUNK_BYTES, &tm_q, q_full, c * C::SW_COLS, w.qpair * kBlockM, w.bh,
                       pol_q);
       }
@@ -457,12 +465,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int i = 0; i < ITERS; ++i) {
             const int key = jt * kBlockN + (ct >> 3) + ROW_STEP * i;
-            e[i] = key < p.N ? ld_nc_u8(p.v_sf + (head_row0 + key) * 4 + blk_d) : 0xFFFFu;
+            e[i] = key < p.N && sf_row_ok(p, head_row0 + key) ? ld_nc_u8(p.v_sf + (head_row0 + key) * 4 + blk_d)
+                                                              : 0xFFFFu;
           }
         };
         uint32_t e_next[ITERS];
         load_e(0, e_next);
-        const int sv = static_cast<int>((head_sf_max(p.v_sf, head_row0, kend, lane) >> (8 * blk_d)) & 0xFFu);
+        const uint32_t vmax = sf_row_ok(p, head_row0 + kend - 1) ? head_sf_max(p.v_sf, head_row0, kend, lane) : 0u;
+        const int sv = static_cast<int>((vmax >> (8 * blk_d)) & 0xFFu);
         for (int j = 0; j < nkv; ++j, ++vb) {
           const uint32_t vg = g + 2 * j + 1, vslot = vg % C::NSLOT, b = vb & 1;
           uint32_t e_cur[ITERS];
@@ -522,7 +532,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
         const int rr = row0 + 32 * h + lane;
-        wv[h] = rr < p.N ? ld_nc_u32(reinterpret_cast<const uint32_t*>(sf) + hrow0 + rr) : 0x7F7F7F7Fu;
+        wv[h] = rr < p.N && sf_row_ok(p, hrow0 + rr) ? ld_nc_u32(reinterpret_cast<const uint32_t*>(sf) + hrow0 + rr)
+                                                      : 0x7F7F7F7Fu;
       }
     };
     auto sf_store = [&](const uint8_t* sf, size_t hrow0, int row0, uint32_t col) {
@@ -584,7 +595,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int key = j * kBlockN + lane + 32 * i;
-            vw[i] = key < p.N ? ld_nc_u32(reinterpret_cast<const uint32_t*>(p.v_sf) + head_row0 + key) : 0u;
+            vw[i] = key < p.N && sf_row_ok(p, head_row0 + key)
+                        ? ld_nc_u32(reinterpret_cast<const uint32_t*>(p.v_sf) + head_row0 + key)
+                        : 0u;
           }
           if (j + 2 < nkv)
             sf_load(p.k_sf, head_row0, (j + 2) * kBlockN, wa);
@@ -666,8 +679,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
         for (int b = 0; b < 4; ++b) f_blk[b] = inv_l * f32_pow2(static_cast<int>((v_sfmax >> (8 * b)) & 0xFFu) - 134);
       }
-      const bool in_range = row < p.N;
-      __nv_bfloat16* orow = p.o + (head_row0 + (in_range ? row : 0)) * C::D;
+      const size_t grow = head_row0 + row;   // row over all heads
+      const bool in_range = row < p.N && dbg_ok(grow < p.out_rows, kSiteFwd1Out, grow);
+      __nv_bfloat16* orow = p.o + (in_range ? grow : 0) * C::D;
 #pragma unroll
       for (int cb = 0; cb < C::D; cb += 32) {
         const float f = f_blk[(cb / 32) & 3];
@@ -685,7 +699,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
         }
       }
-      if (p.lse != nullptr && in_range) p.lse[head_row0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (p.lse != nullptr && in_range) p.lse[grow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
       blk += nkv;
       u = un;
       kc = kn;

@@ -136,6 +136,7 @@ struct FwdParams {
   const float* v_scale;
   uint64_t timeout_cycles;  // per pipeline wait, in SM cycles
   int fault_unit;           // testing only: the producer withholds this unit's first K tile (-1: none)
+  uint32_t out_rows;        // rows of O and LSE the kernel may write (BH * N); checked in debug builds
 };
 
 // Bounded wait that ignores the abort word (used only while draining after an
@@ -391,8 +392,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (q_loads > 0 && !(ok = wait_all(q_empty, (q_loads - 1) & 1))) break;
       if (elect_one()) {
         mbar_arrive_expect_tx(q_full, C::Q_TILES * C::TILE_BYTES);
+        // (debug) a unit outside the launch's heads or Q tiles loads nothing
+        const bool unit_ok = dbg_ok(w.bh < p.BH && w.qpair * C::Q_TILES * kBlockM < p.N, kSiteTmaCoord,
+                                    static_cast<unsigned>(u));
 #pragma unroll
-        for (int t = 0; t < C::Q_TILES; ++t)
+        for (int t = 0; t < C::Q_TILES && unit_ok; ++t)
 #pragma unroll
           for (int c = 0; c < C::CHUNKS; ++c)
             tma_load_3d(smem + C::SMEM_Q + t * C::TILE_BYTES + c * C::CHUNK_BYTES, &tm_q, q_full, c * C::SW_COLS,
@@ -719,8 +723,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_fence_after();
       float inv_l = 1.f / l_run;
       if constexpr (C::FP8) inv_l *= v_max;   // undo the V ratio folded into P
-      const bool in_range = row < p.N;
-      __nv_bfloat16* orow = p.o + (static_cast<size_t>(bh) * p.N + (in_range ? row : 0)) * C::D;
+      const size_t grow = static_cast<size_t>(bh) * p.N + row;   // row over all heads
+      const bool in_range = row < p.N && dbg_ok(grow < p.out_rows, kSiteFwdOut, grow);
+      __nv_bfloat16* orow = p.o + (in_range ? grow : 0) * C::D;
 #pragma unroll
       for (int cb = 0; cb < C::D; cb += 32) {
         uint32_t ov[32];
@@ -737,8 +742,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
         }
       }
-      if (p.lse != nullptr && in_range)
-        p.lse[static_cast<size_t>(bh) * p.N + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (p.lse != nullptr && in_range) p.lse[grow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
     if (!ok) record_timeout();
   }

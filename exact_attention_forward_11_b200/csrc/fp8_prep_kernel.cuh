@@ -278,7 +278,8 @@ __global__ void __launch_bounds__(PrepCfg::THREADS, 1)
           const int bh = tile / T, t = tile % T;
           tma_store_3d(&tm_out, smem + C::SMEM_OUT + ob * C::OUT_BYTES, 0, t * kPrepTile, bh);
           bulk_commit_group();
-          scales[static_cast<size_t>(bh) * T + t] = sc;
+          if (dbg_ok(tile < num_tiles, kSiteFp8Scale, static_cast<unsigned>(tile)))
+            scales[static_cast<size_t>(bh) * T + t] = sc;
           // the previous store has read its staging tile: free it
           if (i >= 1) {
             bulk_wait_group_read<1>();

@@ -25,6 +25,7 @@
 #include <cuda_bf16.h>
 
 #include "sm100.cuh"
+#include "status.cuh"
 
 namespace attn {
 
@@ -73,7 +74,7 @@ __global__ void __launch_bounds__(kMxQuantThreads)
       amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
       const int e = mx_block_exponent(amax);
       const float inv = __int_as_float((127 - e) << 23);   // 2^-E, E in [-127, 119]: a normal fp32
-      if (b < nblk) {
+      if (b < nblk && dbg_ok(b >= 0, kSiteMxBlock, static_cast<unsigned long long>(b))) {
         const uint32_t lo = b200::pack_e4m3x4(v[0] * inv, v[1] * inv, v[2] * inv, v[3] * inv);
         const uint32_t hi = b200::pack_e4m3x4(v[4] * inv, v[5] * inv, v[6] * inv, v[7] * inv);
         *reinterpret_cast<uint2*>(codes + b * 32 + sub * 8) = make_uint2(lo, hi);

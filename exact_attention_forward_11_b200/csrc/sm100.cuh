@@ -7,6 +7,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "status.cuh"
+
 namespace b200 {
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -81,10 +83,17 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
 
+// Every x coordinate this library issues is a multiple of 16 elements (so it
+// starts on a 16-byte boundary for every element size); debug builds check
+// that, and that stores start at non-negative coordinates, and skip a copy that
+// breaks it (a skipped load then leaves its barrier incomplete, and the bounded
+// wait on it ends the CTA with a timeout).
+
 // 3-D tiled bulk tensor load global -> shared, completion counted in bytes on
 // `bar`. Coordinates are {x (innermost), y, z}. No multicast.
 __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
                                             int z, uint64_t cache_policy) {
+  if (!attn::dbg_ok((x & 15) == 0, attn::kSiteTmaCoord, static_cast<unsigned>(x))) return;
   asm volatile(
       "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
       " [%0], [%1, {%3, %4, %5}], [%2], %6;" ::"r"(smem_addr(dst)),
@@ -95,6 +104,7 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 // 3-D tiled bulk tensor store shared -> global, tracked by the issuing
 // thread's bulk async-group. Elements outside the tensor are not written.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+  if (!attn::dbg_ok((x & 15) == 0 && y >= 0 && z >= 0, attn::kSiteTmaCoord, static_cast<unsigned>(x))) return;
   asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
                "r"(smem_addr(src)), "r"(x), "r"(y), "r"(z)

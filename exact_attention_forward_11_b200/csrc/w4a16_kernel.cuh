@@ -257,6 +257,7 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     } else if (h == 0) {
       tc_fence_after();
       __half* ycol = p.y + n0 + t;
+      const bool col_ok = dbg_ok(n0 + t < p.N, kSiteW4Out, static_cast<unsigned>(n0 + t));
       for (int c0 = 0; c0 < mpad; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem_base + lane_off + T_D + c0, v);
@@ -264,7 +265,7 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int m = c0 + i;
-          if (m < p.M) ycol[static_cast<size_t>(m) * p.N] = __float2half_rn(__uint_as_float(v[i]));
+          if (m < p.M && col_ok) ycol[static_cast<size_t>(m) * p.N] = __float2half_rn(__uint_as_float(v[i]));
         }
       }
     }

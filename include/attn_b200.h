@@ -57,7 +57,8 @@ typedef enum {
   ATTN_ERR_UNSUPPORTED = 2,  /* head width or dtype this build has no kernel for */
   ATTN_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned                 */
   ATTN_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed              */
-  ATTN_ERR_TIMEOUT = 5       /* a device pipeline wait ran out (see below)       */
+  ATTN_ERR_TIMEOUT = 5,      /* a device pipeline wait ran out (see below)       */
+  ATTN_ERR_BOUNDS = 6        /* debug builds: a device-side index check failed   */
 } attn_status;
 
 /* Element type of attn_fwd's q, k, v and o (passed as an int-sized enum). */
@@ -231,10 +232,41 @@ ATTN_API attn_status attn_bwd_noalloc(const void* q, const void* k, const void* 
 
 /*
  * attn_get_device_status - synchronises `stream`, then reads and clears the
- * device status word that kernels set when a pipeline wait timed out.
- * Returns ATTN_OK, ATTN_ERR_TIMEOUT, or ATTN_ERR_CUDA if the read failed.
+ * device status word that kernels set when a pipeline wait timed out (or, in
+ * a debug build, when an index check failed).
+ * Returns ATTN_OK, ATTN_ERR_BOUNDS (debug builds: some check failed since the
+ * last read; it takes precedence over a timeout recorded in the same word),
+ * ATTN_ERR_TIMEOUT, or ATTN_ERR_CUDA if the read failed.
  */
 ATTN_API attn_status attn_get_device_status(void* stream);
+
+/*
+ * Debug build (libattn_b200_debug.so, compiled with -DATTN_DEBUG; the pages
+ * define no counterpart: this is the library's own checking aid). Every kernel
+ * then checks, before the access, the row index of each global store of O,
+ * LSE, dQ, dK, dV, FP8 tile scales, MXFP8 codes and scale bytes and W4A16
+ * output columns against the extent the call's sizes give, the row of each
+ * MXFP8 scale-byte load and backward LSE / D_i load, and each TMA coordinate
+ * (x a multiple of 16 elements, stores at non-negative coordinates, work units
+ * inside the launch). A failing check skips the access (nothing traps) and
+ * records ATTN_ERR_BOUNDS in the status word, plus its site and index; a
+ * skipped TMA load leaves its pipeline barrier incomplete, so the launch also
+ * ends through the bounded-wait timeout. Results of a debug build are
+ * bit-identical to the release build's when no check fails.
+ *
+ * attn_debug_build - 1 in a debug build, 0 otherwise.
+ *
+ * attn_debug_last_failure - synchronises `stream`, then reads and clears the
+ * site and index of the first check that failed since the last call (site 0:
+ * none). Sites: 1 O / LSE row (two-Q-tile forward), 2 O / LSE row (one-Q-tile
+ * forward), 3 MXFP8 scale-byte row load, 4 dK / dV row, 5 LSE / D_i load (dK dV
+ * kernel), 6 dQ row and its LSE / D_i load, 7 FP8 tile scale, 8 MXFP8 block,
+ * 9 W4A16 output column, 10 TMA coordinate or work unit. `site` and `index`
+ * are host pointers. Returns ATTN_OK, ATTN_ERR_INVALID_ARG for a null pointer,
+ * or ATTN_ERR_CUDA. In a release build the site is always 0.
+ */
+ATTN_API int attn_debug_build(void);
+ATTN_API attn_status attn_debug_last_failure(int* site, long long* index, void* stream);
 
 /* attn_status_string - static, human-readable name of a status code. */
 ATTN_API const char* attn_status_string(int status);

@@ -1,5 +1,5 @@
 /*
- * attn_b200_testing.h - testing hook of the attention library (not part of the
+ * attn_b200_testing.h - testing hooks of the attention library (not part of the
  * operation; the pages define no counterpart).
  *
  * attn_fwd_inject_timeout - attn_fwd for BF16, d = 128, always on the
@@ -49,6 +49,21 @@ ATTN_API attn_status attn_fwd_one_tile_inject_timeout(const void* q, const void*
                                                       float* lse, int B, int H, int N, int d, float scale,
                                                       int causal, int fault_unit,
                                                       unsigned long long wait_limit_cycles, void* stream);
+
+/*
+ * attn_fwd_debug_row_limit - debug builds only (ATTN_ERR_UNSUPPORTED otherwise):
+ * attn_fwd (BF16, same arguments, same schedule choice) with the kernels told
+ * that O and LSE hold only `row_limit` rows (rows counted over all heads,
+ * b * H * N + h * N + i). The debug checks then reject, skip and record
+ * (ATTN_ERR_BOUNDS, site 1 or 2, index = a rejected row) every store of
+ * a row at or past the limit, while the caller's buffers still hold all
+ * B*H*N rows, so the check can be seen to fire without any access outside
+ * them. Rows below the limit are written as attn_fwd writes them.
+ * 0 <= row_limit <= B*H*N, else ATTN_ERR_INVALID_ARG.
+ */
+ATTN_API attn_status attn_fwd_debug_row_limit(const void* q, const void* k, const void* v, void* o, float* lse,
+                                              int B, int H, int N, int d, float scale, int causal,
+                                              long long row_limit, void* stream);
 
 #ifdef __cplusplus
 }

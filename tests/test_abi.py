@@ -146,3 +146,30 @@ def test_w4a16_argument_validation(lib):
     assert call(6, 200) == lib.ATTN_ERR_UNSUPPORTED       # N not a multiple of 128
     assert call(7, 100) == lib.ATTN_ERR_UNSUPPORTED       # K not a multiple of 128
     assert call(4, FAKE + 2) == lib.ATTN_ERR_MISALIGNED
+
+
+def test_debug_build_exports_the_same_boundary(lib):
+    """The debug build (-DATTN_DEBUG) builds, exports every declared symbol, says
+    it is the debug build, and validates arguments on the host like the release
+    build; the release build refuses the debug-only hook without touching CUDA."""
+    from exact_attention_forward_11_b200 import build
+    so = build.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", so], capture_output=True, text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(declared_symbols()) <= exported
+    assert lib.attn_debug_build() == 0
+    assert lib.attn_status_string(6) == "ATTN_ERR_BOUNDS"
+    assert lib.attn_fwd_debug_row_limit(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 64, 0.0, 0, 4, None) == \
+        lib.ATTN_ERR_UNSUPPORTED
+    prev = lib.use_library(lib.DEBUG_LIB_PATH)
+    try:
+        assert lib.attn_debug_build() == 1
+        f = lib.attn_fwd_debug_row_limit
+        assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 64, 0.0, 0, -1, None) == lib.ATTN_ERR_INVALID_ARG
+        assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 64, 0.0, 0, 9, None) == lib.ATTN_ERR_INVALID_ARG
+        assert f(None, FAKE, FAKE, FAKE, None, 1, 1, 8, 64, 0.0, 0, 4, None) == lib.ATTN_ERR_INVALID_ARG
+        assert f(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 96, 0.0, 0, 4, None) == lib.ATTN_ERR_UNSUPPORTED
+        assert lib.attn_fwd(FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 64, -1.0, 0, 0, None) == lib.ATTN_ERR_INVALID_ARG
+    finally:
+        lib.use_library(prev)
+    assert lib.attn_debug_build() == 0
