@@ -83,18 +83,29 @@ struct Fwd1Cfg {
   static constexpr int P_CHUNKS = ATTN_P_CHUNKS;
   static constexpr float RESCALE_THRESHOLD = 8.0f;
   static constexpr uint32_t POLY_MASK = ATTN_FWD1_POLY_MASK;
-  // MXFP8: 12 warps, the V conversion spread over four warps (6-9), one on each
-  // SM sub-partition next to its softmax warp; warps 10-11 idle. Register split
-  // (launch: 65536 / 384 -> 168 per thread = 64512 in total): softmax warpgroup
-  // 248, the other two warpgroups 128: 128 * 248 + 256 * 128 = 64512.
-  static constexpr int THREADS = MX ? 384 : 256;
+  // MXFP8: 16 warps. The softmax of the Q tile runs on two warpgroups (warps 0-3
+  // and 12-15), warpgroup h taking keys [64 h, 64 h + 64) of every row: one warp
+  // on an SM sub-partition cannot issue exponentials at the MUFU unit's rate,
+  // two warps sharing it can. The two warps of a lane quarter trade their row
+  // maxima (every block) and row sums (every unit) through shared memory and a
+  // bounded mbarrier. The V conversion runs on warps 6-9, one per sub-partition;
+  // warps 10-11 are idle. Register split (launch: 65536 / 512 -> 128 per
+  // thread): softmax warpgroups 176, the other two 80: 2 * 128 * (176 + 80).
+  // BF16: 8 warps, one softmax warpgroup (keys of a row on one thread).
+  static constexpr int SPLIT = MX ? 2 : 1;
+  static constexpr int SOFTMAX_WARP1 = 12;       // first warp of the second softmax warpgroup (SPLIT == 2)
+  static constexpr int THREADS = MX ? 512 : 256;
   static constexpr int PRODUCER_WARP = 4;
   static constexpr int MMA_WARP = 5;
   static constexpr int CONV_WARPS = MX ? 4 : 0;
   static constexpr int CONV_ITERS = MX ? 128 * 8 / (32 * CONV_WARPS) : 1;   // (row, 16-code unit) pairs per thread
-  static constexpr uint32_t REGS_SOFTMAX = 248;
-  static constexpr uint32_t REGS_OTHER = 128;
-  static_assert(!MX || 128 * REGS_SOFTMAX + 256 * REGS_OTHER <= 168 * THREADS, "register split");
+  static constexpr uint32_t REGS_SOFTMAX = 176;
+  static constexpr uint32_t REGS_OTHER = 80;
+  static_assert(!MX || 2 * 128 * (REGS_SOFTMAX + REGS_OTHER) <= 65536, "register split");
+  static_assert(SPLIT == 1 || ATTN_P_CHUNKS == 2, "one P chunk per softmax warpgroup");
+  // TMEM column of P chunk c inside its S buffer: P chunk c (keys 64 c ..) lies over
+  // the S columns of the warpgroup that writes it
+  static constexpr uint32_t P_COL_STEP = SPLIT == 2 ? 64 : 32;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t O_COL0 = 256;
   static constexpr uint32_t SFA_COL = 384;
@@ -107,10 +118,11 @@ struct Fwd1Cfg {
   static constexpr int SMEM_VCONV = SMEM_KV + NSLOT * TILE_BYTES;
   static constexpr int SMEM_BAR = SMEM_VCONV + VCONV_BUFS * VCONV_BYTES;
   // q_full, q_empty, kv_full[NSLOT], kv_empty[NSLOT], s_full[2], p_full[2][P_CHUNKS],
-  // pv_done[2], sfb_ready[2], vconv_full[2], vconv_empty[2], drain
-  static constexpr int NUM_BARS = 2 + 2 * NSLOT + 2 + 2 * P_CHUNKS + 2 + 2 + 2 + 2 + 1;
-  static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;
-  static constexpr int SMEM_BYTES = SMEM_MISC + 16 + 1024;
+  // pv_done[2], sfb_ready[2], vconv_full[2], vconv_empty[2], drain, xch[4], sv_ready[4]
+  static constexpr int NUM_BARS = 2 + 2 * NSLOT + 2 + 2 * P_CHUNKS + 2 + 2 + 2 + 2 + 1 + 4 + 4;
+  static constexpr int SMEM_MISC = SMEM_BAR + NUM_BARS * 8;    // TMEM address, abort word, sv words [4]
+  static constexpr int SMEM_XCH = SMEM_MISC + 32;              // [2 slots][2 warpgroups][128 rows] fp32
+  static constexpr int SMEM_BYTES = SMEM_XCH + (SPLIT > 1 ? 2 * 2 * 128 * 4 : 0) + 1024;
   static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 };
 
@@ -217,6 +229,23 @@ __device__ __forceinline__ uint32_t head_sf_max(const uint8_t* sf, size_t head_r
   return m;
 }
 
+// One softmax warpgroup's share of a row (64 keys, SPLIT == 2): P = 2^(s c - m)
+// as 16-bit pairs into TMEM at p_tm, released to the MMA thread on `bar`;
+// returns the fp32 sum of the share.
+template <class C>
+__device__ __forceinline__ float p_share_to_tmem(const uint32_t (&sr)[64], float c, float m, uint32_t p_tm,
+                                                 uint64_t* bar) {
+  using namespace b200;
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+  uint32_t pk[32];
+  p_chunk_bf16<0u, 32, C::PV_F16>(sr, 0, c, m, acc, pk);
+  tmem_st32(p_tm, pk);
+  release_chunk(bar);
+  float a, b;
+  f2_unpack(f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3])), a, b);
+  return a + b;
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     attn_fwd1_sm100(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -236,8 +265,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* vconv_full = sfb_ready + 2;              // 2: MX f16 V tile written (2 converter warps)
   uint64_t* vconv_empty = vconv_full + 2;            // 2: its P V done (MMA commit)
   uint64_t* drain_bar = vconv_empty + 2;
+  uint64_t* xch = drain_bar + 1;                     // 4: the two softmax warps of a lane quarter traded values
+  uint64_t* sv_ready = xch + 4;                      // 4: MX, a unit's V scale maxima written (converter warp)
+  float* xbuf = reinterpret_cast<float*>(smem + C::SMEM_XCH);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::SMEM_MISC);
   uint32_t* abort_word = tmem_slot + 1;
+  uint32_t* sv_word = tmem_slot + 4;                 // 4 slots (unit index mod 4)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -259,6 +292,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(vconv_empty + b, 1);
     }
     mbar_init(drain_bar, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(xch + q, 2);
+      mbar_init(sv_ready + q, 1);
+    }
     *abort_word = 0u;
     fence_barrier_init();
     fence_proxy_async_shared();
@@ -380,8 +417,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
       for (int i = 0; i < STEPS; ++i) {
         const int kv = c * STEPS + i;
-        mma_f16_ts(tmem_base + C::O_COL0, tmem_base + b * 128 + kv * 8, smem_desc(va + ((kv * 16 * 128) >> 4), hi),
-                   idesc_o, (acc || i > 0) ? 1u : 0u, leader);
+        mma_f16_ts(tmem_base + C::O_COL0, tmem_base + b * 128 + c * C::P_COL_STEP + i * 8,
+                   smem_desc(va + ((kv * 16 * 128) >> 4), hi), idesc_o, (acc || i > 0) ? 1u : 0u, leader);
       }
     };
     uint32_t g = 0, blk = 0, vb = 0;
@@ -439,7 +476,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     commit(drain_bar);
     drain_wait(drain_bar, 0, p.timeout_cycles);
     __syncwarp();
-  } else if (warp > C::MMA_WARP) {
+  } else if (warp > C::MMA_WARP && (C::SPLIT == 1 || warp < C::SOFTMAX_WARP1)) {
     if constexpr (C::MX) {
       regs_decrease<C::REGS_OTHER>();
     }
@@ -452,7 +489,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       constexpr int ROW_STEP = 4 * C::CONV_WARPS;
       const int ct = (warp - C::MMA_WARP - 1) * 32 + lane;
       const int un = ct & 7, blk_d = un >> 1;
-      uint32_t g = 0, vb = 0;
+      uint32_t g = 0, vb = 0, cu = 0;
       int kc;
       for (int u = find_unit(0, kc); ok && u >= 0; u = find_unit(kc + 1, kc)) {
         const UnitInfo<C> w(up, u, QB, QB);
@@ -473,6 +510,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         load_e(0, e_next);
         const uint32_t vmax = sf_row_ok(p, head_row0 + kend - 1) ? head_sf_max(p.v_sf, head_row0, kend, lane) : 0u;
         const int sv = static_cast<int>((vmax >> (8 * blk_d)) & 0xFFu);
+        // the softmax scales O column block b by 2^(sv_b - 134) in the unit's
+        // epilogue: the first converter warp hands the word over (slot = unit
+        // index mod 4; the converters run at most two units ahead of the softmax)
+        if (warp == C::MMA_WARP + 1 && lane == 0) {
+          sv_word[cu & 3] = vmax;
+          mbar_arrive(sv_ready + (cu & 3));
+        }
+        ++cu;
         for (int j = 0; j < nkv; ++j, ++vb) {
           const uint32_t vg = g + 2 * j + 1, vslot = vg % C::NSLOT, b = vb & 1;
           uint32_t e_cur[ITERS];
@@ -520,19 +565,44 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       if (!ok && lane == 0) record_timeout();
     }
   } else {
-    // ======================= softmax: one thread per query row =======================
+    // ======================= softmax: one thread per (query row, key share) =======================
+    // Warpgroup h (SPLIT of them) takes keys [NCOL h, NCOL h + NCOL) of row
+    // 32 (warp % 4) + lane and writes P chunk h over its own S columns. The first
+    // warpgroup (lead) also keeps the MX scale factors in TMEM, rescales O and
+    // writes LSE; each warpgroup writes its share of the O columns.
     if constexpr (C::MX) regs_increase<C::REGS_SOFTMAX>();
-    const int r = warp * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    constexpr int NCOL = 128 / C::SPLIT;           // keys of a block per thread
+    constexpr int OCOL = C::D / C::SPLIT;          // output columns per thread
+    const int h = (C::SPLIT > 1 && warp >= C::SOFTMAX_WARP1) ? 1 : 0;
+    const bool lead = h == 0;
+    const int wq = warp & 3;                       // lane quarter of TMEM this warp may access
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t o_tm = tmem_base + lane_off + C::O_COL0;
-    // MX scale factors into TMEM: this warp's lane quarter gets, in column col + h,
-    // the scale word of row row0 + 32 h + lane (rows past N: 0x7F bytes, scale 1).
+    // (SPLIT == 2) value of this row from the other warpgroup: both warps of the
+    // lane quarter write theirs, arrive, and wait with the bounded waiter; the two
+    // slots alternate, so a slot is rewritten only after the partner has passed
+    // the exchange that followed its read. Sets ok = false when the wait gives up.
+    uint32_t xc = 0;
+    auto exchange = [&](float v) -> float {
+      float* xb = xbuf + (xc & 1u) * 256;
+      xb[h * 128 + r] = v;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(xch + wq);
+      ok = wait_all(xch + wq, xc & 1u);
+      tc_fence_after();
+      ++xc;
+      return xb[(h ^ 1) * 128 + r];
+    };
+    // MX scale factors into TMEM: this warp's lane quarter gets, in column col + q,
+    // the scale word of row row0 + 32 q + lane (rows past N: 0x7F bytes, scale 1).
     // The loads are issued ahead of the waits they would otherwise stall.
     auto sf_load = [&](const uint8_t* sf, size_t hrow0, int row0, uint32_t (&wv)[4]) {
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const int rr = row0 + 32 * h + lane;
-        wv[h] = rr < p.N && sf_row_ok(p, hrow0 + rr) ? ld_nc_u32(reinterpret_cast<const uint32_t*>(sf) + hrow0 + rr)
+      for (int q = 0; q < 4; ++q) {
+        const int rr = row0 + 32 * q + lane;
+        wv[q] = rr < p.N && sf_row_ok(p, hrow0 + rr) ? ld_nc_u32(reinterpret_cast<const uint32_t*>(sf) + hrow0 + rr)
                                                       : 0x7F7F7F7Fu;
       }
     };
@@ -552,10 +622,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
     };
     uint32_t blk = 0;
+    uint32_t su = 0;   // units so far (MX: slot and phase of sv_ready)
     int kc;
     int u = find_unit(0, kc);
     if constexpr (C::MX) {
-      if (u >= 0) {
+      if (u >= 0 && lead) {
         const UnitInfo<C> w(up, u, QB, QB);
         const size_t hrow0 = static_cast<size_t>(w.bh) * p.N;
         sf_store(p.q_sf, hrow0, w.qpair * kBlockM, C::SFA_COL);
@@ -581,70 +652,71 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const size_t next_row0 = static_cast<size_t>(bh_next) * p.N;
       const uint32_t L = blk + nkv - 1;   // the unit's last global block
       float m_run = __int_as_float(0xff800000u);
-      float l_run = 0.f;
-      uint32_t v_sfmax = 0u;   // MX: byte-wise max of the V scale words of the key rows this lane passed
+      float l_run = 0.f;                  // this thread's share of the row sum
       for (int j = 0; j < nkv; ++j) {
         const uint32_t B = blk + j, bj = B & 1, ph = (B >> 1) & 1;
         const uint32_t s_tm = tmem_base + lane_off + bj * 128;
         // MX: the K scale words this iteration stores (block j + 2, or the next
-        // unit's block 0) and the V scale words of key rows
-        // j*128 + lane + 32 i (the warp passes every key row of the tile), loaded
-        // before the S wait so that their latency hides behind it
-        uint32_t wa[4], vw[4];
+        // unit's block 0), loaded before the S wait so that their latency hides
+        // behind it
+        uint32_t wa[4];
         if constexpr (C::MX) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int key = j * kBlockN + lane + 32 * i;
-            vw[i] = key < p.N && sf_row_ok(p, head_row0 + key)
-                        ? ld_nc_u32(reinterpret_cast<const uint32_t*>(p.v_sf) + head_row0 + key)
-                        : 0u;
+          if (lead) {
+            if (j + 2 < nkv)
+              sf_load(p.k_sf, head_row0, (j + 2) * kBlockN, wa);
+            else if (un >= 0 && (B + 1 == L || (B == L && nkv == 1)))
+              sf_load(p.k_sf, next_row0, 0, wa);
           }
-          if (j + 2 < nkv)
-            sf_load(p.k_sf, head_row0, (j + 2) * kBlockN, wa);
-          else if (un >= 0 && (B + 1 == L || (B == L && nkv == 1)))
-            sf_load(p.k_sf, next_row0, 0, wa);
         }
         ok = wait_all(s_full + bj, ph);
         if (!ok) break;
         tc_fence_after();
-        uint32_t sr[128];
-        tmem_ld32(s_tm + 0, sr + 0);
-        tmem_ld32(s_tm + 32, sr + 32);
-        tmem_ld32(s_tm + 64, sr + 64);
-        tmem_ld32(s_tm + 96, sr + 96);
-        tmem_ld_wait<128>(sr);
+        uint32_t sr[NCOL];
+#pragma unroll
+        for (int q = 0; q < NCOL / 32; ++q) tmem_ld32(s_tm + NCOL * h + 32 * q, sr + 32 * q);
+        tmem_ld_wait<NCOL>(sr);
         if constexpr (C::MX) {
-          v_sfmax = max_u8x4(max_u8x4(v_sfmax, max_u8x4(vw[0], vw[1])), max_u8x4(vw[2], vw[3]));
           // Every S MMA up to block B is complete: the K scale columns of buffer
           // bj (read by S(B)) take the scales of block B + 2; once S of the unit's
           // last block is read, the Q columns take the next unit's.
-          if (j + 2 < nkv) {
-            tmem_st4(tmem_base + lane_off + C::SFB_COL + 4 * bj, wa);
-            sf_publish(bj, false);
-          } else if (un >= 0) {
-            if (B + 1 == L) tmem_st4(tmem_base + lane_off + C::SFB_COL + 4 * bj, wa);   // next unit's block 0
-            if (B == L) {   // once per unit: these loads are not prefetched
-              sf_store(p.q_sf, next_row0, qb_next * kBlockM, C::SFA_COL);
-              if (nkv == 1) tmem_st4(tmem_base + lane_off + C::SFB_COL + 4 * (bj ^ 1u), wa);
-              if (nkv_next > 1) sf_store(p.k_sf, next_row0, kBlockN, C::SFB_COL + 4 * bj);
-              sf_publish(bj ^ 1u, nkv_next > 1);
+          if (lead) {
+            if (j + 2 < nkv) {
+              tmem_st4(tmem_base + lane_off + C::SFB_COL + 4 * bj, wa);
+              sf_publish(bj, false);
+            } else if (un >= 0) {
+              if (B + 1 == L) tmem_st4(tmem_base + lane_off + C::SFB_COL + 4 * bj, wa);   // next unit's block 0
+              if (B == L) {   // once per unit: these loads are not prefetched
+                sf_store(p.q_sf, next_row0, qb_next * kBlockM, C::SFA_COL);
+                if (nkv == 1) tmem_st4(tmem_base + lane_off + C::SFB_COL + 4 * (bj ^ 1u), wa);
+                if (nkv_next > 1) sf_store(p.k_sf, next_row0, kBlockN, C::SFB_COL + 4 * bj);
+                sf_publish(bj ^ 1u, nkv_next > 1);
+              }
             }
           }
         }
         const float c = p.scale_log2;
         const bool masked = (j == nkv - 1) && (p.causal || (p.N % kBlockN) != 0);
         if (masked) {
-          const int limit = (p.causal ? min(row, p.N - 1) : p.N - 1) - j * kBlockN;   // last visible key
+          // last visible key of this thread's share
+          const int limit = (p.causal ? min(row, p.N - 1) : p.N - 1) - j * kBlockN - NCOL * h;
 #pragma unroll
-          for (int i = 0; i < 128; ++i)
+          for (int i = 0; i < NCOL; ++i)
             if (i > limit) sr[i] = 0xff800000u;
         }
-        const float m_blk = row_max128(sr) * c;
+        float m_blk = row_max<NCOL>(sr) * c;
+        if constexpr (C::SPLIT > 1) {
+          const float m_other = exchange(m_blk);
+          if (!ok) break;
+          m_blk = fmaxf(m_blk, m_other);
+        }
         float m_use = m_run;
         if (m_blk - m_run > C::RESCALE_THRESHOLD) m_use = m_blk;
         const bool moved = m_use != m_run;
         const float alpha = moved ? ex2_approx(m_run - m_use) : 1.f;
-        if (j > 0 && __any_sync(0xffffffffu, moved)) {
+        // Both warpgroups see the same maximum, so they move together. The lead
+        // rescales every column of O before it releases P chunk 0, and the MMA
+        // issues chunk 0 before chunk 1: all of this block's P V follows it.
+        if (lead && j > 0 && __any_sync(0xffffffffu, moved)) {
           // O holds P V up to block B - 1 once that P V has completed
           if (!(ok = wait_all(pv_done + (bj ^ 1u), ((B - 1) >> 1) & 1))) break;
           tc_fence_after();
@@ -659,34 +731,48 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
         }
         uint64_t* pf = p_full + bj * C::P_CHUNKS;
-        const float sum = masked ? p_row_to_tmem<C, 0u>(sr, c, m_use, s_tm, pf)
-                                 : p_row_to_tmem<C, C::POLY_MASK>(sr, c, m_use, s_tm, pf);
+        float sum;
+        if constexpr (C::SPLIT == 1) {
+          sum = masked ? p_row_to_tmem<C, 0u>(sr, c, m_use, s_tm, pf)
+                       : p_row_to_tmem<C, C::POLY_MASK>(sr, c, m_use, s_tm, pf);
+        } else {
+          sum = p_share_to_tmem<C>(sr, c, m_use, s_tm + C::P_COL_STEP * h, pf + h);
+        }
         l_run = l_run * alpha + sum;
         m_run = m_use;
       }
       if (!ok) break;
       // ---- epilogue: the unit's last P V complete, then O / l and LSE. The next
-      // unit's first P V (which overwrites O) waits for this group's P, which
-      // comes after these TMEM loads.
+      // unit's first P V (which overwrites O) waits for the lead's P, which comes
+      // after its own TMEM loads and (through the first exchange of the next
+      // unit) after the other warpgroup's.
       if (!(ok = wait_all(pv_done + (L & 1), (L >> 1) & 1))) break;
       tc_fence_after();
-      const float inv_l = 1.f / l_run;
+      float l_row = l_run;
+      if constexpr (C::SPLIT > 1) {
+        const float l_other = exchange(l_run);
+        if (!ok) break;
+        l_row += l_other;
+      }
+      const float inv_l = 1.f / l_row;
       float f_blk[4] = {inv_l, inv_l, inv_l, inv_l};
       if constexpr (C::MX) {
-        // sv_b over every key row of the unit (the same bytes the converters reduce)
-#pragma unroll
-        for (int s = 16; s > 0; s >>= 1) v_sfmax = max_u8x4(v_sfmax, __shfl_xor_sync(0xffffffffu, v_sfmax, s));
+        // sv_b, the maximum V scale byte of column block b over the unit's key
+        // rows, as the converter warps reduced it for the V widening
+        if (!(ok = wait_all(sv_ready + (su & 3), (su >> 2) & 1))) break;
+        const uint32_t v_sfmax = sv_word[su & 3];
 #pragma unroll
         for (int b = 0; b < 4; ++b) f_blk[b] = inv_l * f32_pow2(static_cast<int>((v_sfmax >> (8 * b)) & 0xFFu) - 134);
       }
+      ++su;
       const size_t grow = head_row0 + row;   // row over all heads
       const bool in_range = row < p.N && dbg_ok(grow < p.out_rows, kSiteFwd1Out, grow);
-      __nv_bfloat16* orow = p.o + (in_range ? grow : 0) * C::D;
+      __nv_bfloat16* orow = p.o + (in_range ? grow : 0) * C::D + OCOL * h;
 #pragma unroll
-      for (int cb = 0; cb < C::D; cb += 32) {
-        const float f = f_blk[(cb / 32) & 3];
+      for (int cb = 0; cb < OCOL; cb += 32) {
+        const float f = f_blk[((OCOL * h + cb) / 32) & 3];
         uint32_t ov[32];
-        tmem_ld32(o_tm + cb, ov);
+        tmem_ld32(o_tm + OCOL * h + cb, ov);
         tmem_ld_wait<32>(ov);
         uint32_t packed[16];
 #pragma unroll
@@ -699,7 +785,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
         }
       }
-      if (p.lse != nullptr && in_range) p.lse[grow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (lead && p.lse != nullptr && in_range) p.lse[grow] = (m_run + __log2f(l_row)) * 0.69314718055994531f;
       blk += nkv;
       u = un;
       kc = kn;
