@@ -646,13 +646,21 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       float m_run = __int_as_float(0xff800000u);   // running max of scale*log2(e)*s, log2 units
       float l_run = 0.f;                           // running normaliser, relative to 2^m_run
       float q_sc = 1.f, v_max = 1.f;
+      float ks_next = 1.f, vs_next = 1.f;          // FP8: block j's K and V tile scales, loaded one block ahead
       if constexpr (C::FP8) {
+        ks_next = p.k_scale[bh * T];
+        vs_next = p.v_scale[bh * T];
         q_sc = p.q_scale[bh * T + qb];
         float vm = 0.f;
         for (int i = 0; i < T; ++i) vm = fmaxf(vm, p.v_scale[bh * T + i]);
         v_max = vm > 0.f ? vm : 1.f;
       }
       for (int j = 0; j < nkv_t; ++j) {
+        const float ks = ks_next, vs = vs_next;
+        if (C::FP8 && j + 1 < nkv_t) {   // issued before the S wait, used one block later
+          ks_next = p.k_scale[bh * T + j + 1];
+          vs_next = p.v_scale[bh * T + j + 1];
+        }
         // TMEM loads/stores below are warp-collective: the whole warp goes on or stops
         ok = __all_sync(0xffffffffu, waiter.wait(s_full + t, sc & 1));
         if (!ok) break;
@@ -671,8 +679,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           // of such a tile are then ~0, as they should be) and the V ratio at
           // or above 2^-64 (its P rounds to zero in E4M3; the fp32 row sum
           // keeps its exact share of the normaliser).
-          c = fmaxf(c * (q_sc * p.k_scale[bh * T + j]), 1e-30f);
-          v_log2_ratio = __log2f(fmaxf(p.v_scale[bh * T + j] / v_max, 5.421010862427522e-20f));
+          c = fmaxf(c * (q_sc * ks), 1e-30f);
+          v_log2_ratio = __log2f(fmaxf(vs / v_max, 5.421010862427522e-20f));
         }
         // masking: causal diagonal block and the ragged last key block
         const bool masked = (j == nkv_t - 1) && (p.causal || (p.N % kBlockN) != 0);
