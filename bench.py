@@ -241,12 +241,16 @@ def gpu_smi_id(dev, local):
 
 
 def sustained_bf16_peak():
-    """The measured bf16 GEMM rate over seconds under the power cap (None if absent)."""
+    """(rate, source): the measured bf16 GEMM rate over seconds under the power cap,
+    else the pool's earlier measurement of it (1.4 PFLOP/s at ~1.3 GHz under the
+    1 kW cap)."""
     path = os.path.join(HERE, "MEASURED_PEAKS.json")
     if os.path.exists(path):
         with open(path) as f:
-            return json.load(f).get("bf16_tflops_sustained")
-    return None
+            v = json.load(f).get("bf16_tflops_sustained")
+        if v:
+            return v, "measured"
+    return 1400.0, "fallback"
 
 
 def measured_peaks():
@@ -668,13 +672,13 @@ def roofline(w, kern_ms, sm_mhz, workload, kernel="attn_fwd_sm100"):
         hw *= ratio
         roof["hw_peak_at_sampled_clock"] = round(hw, 1)
         roof["frac_of_hw_peak_at_sampled_clock"] = round(achieved / hw, 4)
-    sus = sustained_bf16_peak()
-    if sus:
-        # a long timed loop meets the 1 kW power cap (see "clocks"); the sustained
-        # GEMM rate is the same-conditions denominator
-        sus = round(sus * ratio, 1)
-        roof["frac_of_sustained_peak"] = round(achieved / sus, 4)
-        roof["sustained_peak"] = sus
+    sus, sus_src = sustained_bf16_peak()
+    # a long timed loop meets the 1 kW power cap (see "clocks"); the sustained
+    # GEMM rate is the same-conditions denominator
+    sus = round(sus * ratio, 1)
+    roof["frac_of_sustained_peak"] = round(achieved / sus, 4)
+    roof["sustained_peak"] = sus
+    roof["sustained_peak_source"] = f"{sus_src} bf16 sustained" + note
     if w.fp8:
         pb = prep_bytes(w)
         roof["prep"] = {name: {"ms": round(kern_ms[name], 5), "algorithmic_bytes": pb,
