@@ -42,6 +42,8 @@ SIGNATURES = {
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "w4a16_gemm": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "attn_fwd_mxfp8_inject_timeout": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I,
+                                           ctypes.c_ulonglong, _P]),
     "attn_fwd_debug_row_limit": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, ctypes.c_longlong, _P]),
     "attn_debug_build": (_I, []),
     "attn_debug_last_failure": (_I, [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_longlong), _P]),
@@ -126,6 +128,13 @@ def attn_fwd_one_tile_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal,
     """Testing hook (include/attn_b200_testing.h): the one-Q-tile schedule with one K tile withheld."""
     return load().attn_fwd_one_tile_inject_timeout(q, k, v, o, lse, B, H, N, d, scale, causal, fault_unit,
                                                    wait_limit_cycles, stream)
+
+
+def attn_fwd_mxfp8_inject_timeout(q8, k8, v8, q_sf, k_sf, v_sf, o, lse, B, H, N, d, scale, causal, fault_unit,
+                                  wait_limit_cycles, stream):
+    """Testing hook (include/attn_b200_testing.h): attn_fwd_mxfp8 with one K tile withheld."""
+    return load().attn_fwd_mxfp8_inject_timeout(q8, k8, v8, q_sf, k_sf, v_sf, o, lse, B, H, N, d, scale, causal,
+                                                fault_unit, wait_limit_cycles, stream)
 
 
 def attn_fwd_debug_row_limit(q, k, v, o, lse, B, H, N, d, scale, causal, row_limit, stream):

@@ -505,9 +505,15 @@ attn_status attn_quantize_mxfp8(const void* x, void* codes, void* sf, int B, int
   return ATTN_OK;
 }
 
-attn_status attn_fwd_mxfp8(const void* q8, const void* k8, const void* v8, const void* q_sf, const void* k_sf,
-                           const void* v_sf, void* o, float* lse, int B, int H, int N, int d, float scale,
-                           int causal, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// attn_fwd_mxfp8's argument checks and launch; fault_unit / wait_limit are the
+// testing hook's (-1 / the normal limit otherwise).
+attn_status fwd_mxfp8(const void* q8, const void* k8, const void* v8, const void* q_sf, const void* k_sf,
+                      const void* v_sf, void* o, float* lse, int B, int H, int N, int d, float scale, int causal,
+                      void* stream, int fault_unit, uint64_t wait_limit) {
   if (q8 == nullptr || k8 == nullptr || v8 == nullptr || o == nullptr || q_sf == nullptr || k_sf == nullptr ||
       v_sf == nullptr)
     return ATTN_ERR_INVALID_ARG;
@@ -519,7 +525,26 @@ attn_status attn_fwd_mxfp8(const void* q8, const void* k8, const void* v8, const
       !aligned16(v_sf) || !aligned16(o) || (lse != nullptr && !aligned16(lse)))
     return ATTN_ERR_MISALIGNED;
   return launch_fwd1<128, true>(q8, k8, v8, o, lse, q_sf, k_sf, v_sf, B * H, N, scale, causal,
-                                static_cast<cudaStream_t>(stream));
+                                static_cast<cudaStream_t>(stream), fault_unit, wait_limit);
+}
+
+}  // namespace
+
+extern "C" {
+
+attn_status attn_fwd_mxfp8(const void* q8, const void* k8, const void* v8, const void* q_sf, const void* k_sf,
+                           const void* v_sf, void* o, float* lse, int B, int H, int N, int d, float scale,
+                           int causal, void* stream) {
+  return fwd_mxfp8(q8, k8, v8, q_sf, k_sf, v_sf, o, lse, B, H, N, d, scale, causal, stream, -1, kWaitLimitCycles);
+}
+
+attn_status attn_fwd_mxfp8_inject_timeout(const void* q8, const void* k8, const void* v8, const void* q_sf,
+                                          const void* k_sf, const void* v_sf, void* o, float* lse, int B, int H,
+                                          int N, int d, float scale, int causal, int fault_unit,
+                                          unsigned long long wait_limit_cycles, void* stream) {
+  if (fault_unit < 0 || wait_limit_cycles < 1024) return ATTN_ERR_INVALID_ARG;
+  return fwd_mxfp8(q8, k8, v8, q_sf, k_sf, v_sf, o, lse, B, H, N, d, scale, causal, stream, fault_unit,
+                   wait_limit_cycles);
 }
 
 attn_status attn_quantize_fp8(const void* x, const void* rot, void* x8, float* scales, int B, int H, int N, int d,

@@ -51,6 +51,23 @@ ATTN_API attn_status attn_fwd_one_tile_inject_timeout(const void* q, const void*
                                                       unsigned long long wait_limit_cycles, void* stream);
 
 /*
+ * attn_fwd_mxfp8_inject_timeout - attn_fwd_mxfp8 (same arguments, same kernel)
+ * with the same planted failure: the producer of work unit `fault_unit` (one
+ * head and one 128-row Q tile, numbered as for attn_fwd_one_tile_inject_timeout)
+ * never loads that unit's first K tile, and every pipeline wait gives up after
+ * `wait_limit_cycles`. Besides the producer / MMA / softmax waits this runs out
+ * the MXFP8 kernel's own: the converter warps' V-tile waits, the exchange of
+ * half-row maxima and sums between its two softmax warpgroups, and the hand-over
+ * of a unit's V scale maxima. fault_unit >= 0 and wait_limit_cycles >= 1024
+ * (else ATTN_ERR_INVALID_ARG); other results as for attn_fwd_inject_timeout.
+ */
+ATTN_API attn_status attn_fwd_mxfp8_inject_timeout(const void* q8, const void* k8, const void* v8,
+                                                   const void* q_sf, const void* k_sf, const void* v_sf, void* o,
+                                                   float* lse, int B, int H, int N, int d, float scale, int causal,
+                                                   int fault_unit, unsigned long long wait_limit_cycles,
+                                                   void* stream);
+
+/*
  * attn_fwd_debug_row_limit - debug builds only (ATTN_ERR_UNSUPPORTED otherwise):
  * attn_fwd (BF16, same arguments, same schedule choice) with the kernels told
  * that O and LSE hold only `row_limit` rows (rows counted over all heads,

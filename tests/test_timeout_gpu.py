@@ -109,3 +109,52 @@ def test_one_tile_starved_unit_times_out_and_context_survives(cuda_lib):
     o_ref, _ = attention_fp64(q.double().numpy(), k.double().numpy(), v.double().numpy(), scale, False,
                               rows=np.arange(768, 896))
     assert np.abs(o.float().cpu().numpy()[0, 1, 768:896] - o_ref[0, 1]).max() <= 2e-2
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_mxfp8_starved_unit_times_out_and_context_survives(cuda_lib, causal):
+    """The planted failure in the MXFP8 forward: beyond the producer / MMA waits it
+    runs out the converter warps' waits, the half-row exchange between the two
+    softmax warpgroups and the hand-over of the V scale maxima. Every other unit
+    (one per CTA here) is bit-identical to an ordinary launch, and the next
+    ordinary launch is too."""
+    lib = cuda_lib
+    dev = torch.device("cuda:0")
+    B, H, N, d = 1, 4, 1024, 128          # 4 heads x 8 Q tiles = 32 units, one per CTA
+    q, k, v = (x.to(dev) for x in _inputs(B, H, N, d, seed=2027))
+    (q8, qs), (k8, ks), (v8, vs) = (lib.quantize_mxfp8(x) for x in (q, k, v))
+    o_ref, lse_ref = lib.forward_mxfp8(q8, k8, v8, qs, ks, vs, causal=causal)
+    torch.cuda.synchronize()
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+
+    o = torch.full((B, H, N, d), float("nan"), dtype=torch.bfloat16, device=dev)
+    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=dev)
+    # unit 5: non-causal, tile 7 - 5 // 4 of head 5 % 4 (rows 768..895 of head 1); causal
+    # units are numbered the same way (heaviest tiles first), so also rows 768..895 of head 1
+    fault_unit, h_f, rows_f = 5, 1, slice(768, 896)
+    t0 = time.time()
+    st = lib.attn_fwd_mxfp8_inject_timeout(q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), qs.data_ptr(),
+                                           ks.data_ptr(), vs.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, N, d,
+                                           0.0, int(causal), fault_unit, WAIT_LIMIT, None)
+    assert st == lib.ATTN_OK, lib.attn_status_string(st)
+    assert lib.attn_get_device_status(None) == lib.ATTN_ERR_TIMEOUT
+    assert time.time() - t0 < 30.0
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+
+    keep = torch.ones((B, H, N), dtype=torch.bool, device=dev)
+    keep[0, h_f, rows_f] = False
+    assert torch.equal(o[keep].view(torch.int16), o_ref[keep].view(torch.int16))
+    assert torch.equal(lse[keep], lse_ref[keep])
+
+    o2, lse2 = lib.forward_mxfp8(q8, k8, v8, qs, ks, vs, causal=causal)
+    torch.cuda.synchronize()
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+    assert torch.equal(o2.view(torch.int16), o_ref.view(torch.int16)) and torch.equal(lse2, lse_ref)
+
+
+def test_mxfp8_inject_timeout_validates_arguments(cuda_lib):
+    lib = cuda_lib
+    f = lib.attn_fwd_mxfp8_inject_timeout
+    assert f(16, 16, 16, 16, 16, 16, 16, 16, 1, 1, 128, 128, 0.0, 0, -1, WAIT_LIMIT, None) == lib.ATTN_ERR_INVALID_ARG
+    assert f(16, 16, 16, 16, 16, 16, 16, 16, 1, 1, 128, 128, 0.0, 0, 0, 100, None) == lib.ATTN_ERR_INVALID_ARG
+    assert f(None, 16, 16, 16, 16, 16, 16, 16, 1, 1, 128, 128, 0.0, 0, 0, WAIT_LIMIT, None) == lib.ATTN_ERR_INVALID_ARG
