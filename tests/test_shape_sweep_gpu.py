@@ -1,5 +1,5 @@
-"""A seeded sweep of random shapes through every forward entry point, against the
-fp64 oracle.
+"""A seeded sweep of random shapes through every forward entry point, the backward
+and the W4A16 GEMM, against the fp64 oracle.
 
 The fixed shape lists of the other parity tests pick the edge cases by hand. This
 sweep draws B, H, N (1 .. 700) and the head width at random from a fixed seed,
@@ -10,7 +10,8 @@ one- and two-tile schedules. Outputs are NaN-prefilled and fenced by canaries;
 the device status word must read ATTN_OK after every launch. Tolerances as in the
 other parity tests: BF16 and MXFP8 max |O - O_ref| <= 2e-2, mean <= 2e-3, FP8
 max <= 1e-1, LSE within 1e-3 (the quantised paths against the oracle run on the
-oracle's own dequantised values).
+oracle's own dequantised values); the backward and W4A16 bounds are those of their
+own tests.
 """
 import math
 
@@ -143,3 +144,65 @@ def test_mxfp8_random_shape(cuda_lib, shape):
     deq = [mx_dequantize(*mx_quantize(x.to(torch.float64).numpy())) for x in (q, k, v)]
     o_ref, lse_ref = attention_fp64(*deq, 1 / math.sqrt(d), causal, rows=rows)
     _check(o, lse, o_ref, lse_ref, rows, TOL_MAX, TOL_MEAN)
+
+
+# ---------------------------------------------------------------- backward and W4A16
+BWD_SHAPES = _draw(10, 20261206, (64, 128))
+
+
+@pytest.mark.parametrize("shape", [(B, H, min(N, 520), d, c) for B, H, N, d, c in BWD_SHAPES], ids=_ids)
+def test_bwd_random_shape(cuda_lib, shape):
+    """The backward through attn_bwd, with the tolerance the backward tests derive
+    (largest element error 2 % of the tensor's largest magnitude, Frobenius 1 %)."""
+    from oracle import attention_bwd_fp64
+    lib = cuda_lib
+    B, H, N, d, causal = shape
+    q, k, v = workloads.make_qkv(B, H, N, d, seed=N * 5 + d + 1)
+    gen = torch.Generator().manual_seed(N + 17)
+    dout = torch.randn((B, H, N, d), generator=gen).to(torch.bfloat16)
+    qd, kd, vd, dod = (x.to(DEV) for x in (q, k, v, dout))
+    o, lse = lib.forward(qd, kd, vd, causal=causal)
+    grads = [Guarded((B, H, N, d), torch.bfloat16) for _ in range(3)]
+    lib.backward(qd, kd, vd, o, lse, dod, causal=causal, dq=grads[0].t, dk=grads[1].t, dv=grads[2].t)
+    torch.cuda.synchronize()
+    assert all(g.intact() for g in grads), "write outside a gradient"
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+    want = attention_bwd_fp64(*(x.to(torch.float64).numpy() for x in (q, k, v, dout)), 1 / math.sqrt(d), causal)
+    for g, ref, name in zip(grads, want, ("dq", "dk", "dv")):
+        got = g.t.float().cpu().numpy()
+        assert np.isfinite(got).all(), f"{name}: NaN/inf (unwritten element?)"
+        err = np.abs(got - ref)
+        assert err.max() <= 2e-2 * np.abs(ref).max() + 1e-5, f"{name}: max err {err.max()}"
+        assert np.linalg.norm(got - ref) <= 1e-2 * np.linalg.norm(ref) + 1e-5 * np.sqrt(ref.size), name
+
+
+def _draw_gemm(n, seed):
+    rng = np.random.default_rng(seed)
+    return [(int(rng.integers(1, 129)), 128 * int(rng.integers(1, 9)), 128 * int(rng.integers(1, 7)))
+            for _ in range(n)]
+
+
+@pytest.mark.parametrize("M,K,N", _draw_gemm(8, 20261207))
+def test_w4a16_random_shape(cuda_lib, M, K, N):
+    """W4A16 GEMM of random M (1 .. 128), K and N (multiples of 128), against the
+    fp64 product of the dequantised weights with the W4A16 tests' element bound
+    (2^-11 relative plus 2^-16 of the sum of |x||w|: fp16 output rounding and fp32
+    accumulation of fp16 products)."""
+    from oracle.w4a16 import dequantize_weights, w4a16_gemm_fp64
+    lib = cuda_lib
+    x, qw, s, z = workloads.make_w4a16(M, N, K, seed=M * 3 + K + N)
+    raw = torch.full((M * N + 2 * CANARY,), float("nan"), dtype=torch.float16, device=DEV)
+    raw[:CANARY] = 5.0
+    raw[-CANARY:] = 5.0
+    y = raw[CANARY:CANARY + M * N].view(M, N)
+    lib.w4a16_matmul(x.to(DEV), qw.to(DEV), s.to(DEV), z.to(DEV), out=y)
+    torch.cuda.synchronize()
+    assert bool((raw[:CANARY] == 5.0).all()) and bool((raw[-CANARY:] == 5.0).all()), "write outside Y"
+    assert lib.attn_get_device_status(None) == lib.ATTN_OK
+    xn, qn, sn, zn = (t.numpy() for t in (x, qw, s, z))
+    ref = w4a16_gemm_fp64(xn, qn, sn, zn)
+    w = dequantize_weights(qn, sn, zn).astype(np.float64)
+    bound = 2.0 ** -11 * np.abs(ref) + 2.0 ** -16 * (np.abs(xn.astype(np.float64)) @ np.abs(w)) + 1e-7
+    got = y.float().cpu().numpy()
+    assert np.isfinite(got).all(), "NaN/inf in Y (unwritten element?)"
+    assert np.all(np.abs(got - ref) <= bound), f"max err {np.abs(got - ref).max()}"
