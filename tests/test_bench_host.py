@@ -78,3 +78,22 @@ def test_reference_arm_prints_one_contract_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["config"]["workload"] == "llm_train_causal"
+
+
+def test_loop_steps_sizing():
+    """Timed loops: the caller's count when given, else at least `minimum` steps
+    and enough for the target duration (so short kernels still span several clock
+    samples and the sustained loop reaches the power-capped regime)."""
+    assert bench.loop_steps(7, 0.5, 10.0, 20) == 7
+    assert bench.loop_steps(None, 0.55, 10.0, 20) == 20          # 20 x 0.55 ms >= 10 ms
+    assert bench.loop_steps(None, 0.041, 10.0, 20) == 244        # ViT batch: ceil(10 / 0.041)
+    assert bench.loop_steps(None, 0.55, 300.0, 500) == 546
+    assert bench.loop_steps(None, 0.0, 10.0, 20) == 100000       # a zero estimate is floored, not divided by
+    assert bench.loop_steps(0, 0.55, 300.0, 500) == 0             # an explicit 0 skips the loop
+
+
+def test_sustained_denominator_fallback(monkeypatch, tmp_path):
+    monkeypatch.setattr(bench, "HERE", str(tmp_path))
+    assert bench.sustained_bf16_peak() == (1400.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"bf16_tflops": 1663.5, "bf16_tflops_sustained": 1410.5}')
+    assert bench.sustained_bf16_peak() == (1410.5, "measured")
