@@ -42,6 +42,8 @@ SIGNATURES = {
     "attn_bwd_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "attn_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "w4a16_gemm": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P]),
+    "w4a16_gemm_splitk": (_I, [_P, _P, _P, _P, _P, _P, ctypes.c_size_t, _I, _I, _I, _P]),
+    "w4a16_gemm_splitk_workspace_bytes": (ctypes.c_size_t, [_I, _I, _I]),
     "attn_fwd_mxfp8_inject_timeout": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _I,
                                            ctypes.c_ulonglong, _P]),
     "attn_fwd_debug_row_limit": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, ctypes.c_longlong, _P]),
@@ -108,6 +110,14 @@ def w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream):
     return load().w4a16_gemm(x, qweight, scales, zeros, y, M, N, K, stream)
 
 
+def w4a16_gemm_splitk(x, qweight, scales, zeros, y, workspace, workspace_bytes, M, N, K, stream):
+    return load().w4a16_gemm_splitk(x, qweight, scales, zeros, y, workspace, workspace_bytes, M, N, K, stream)
+
+
+def w4a16_gemm_splitk_workspace_bytes(M, N, K):
+    return load().w4a16_gemm_splitk_workspace_bytes(M, N, K)
+
+
 def attn_bwd_noalloc(q, k, v, o, lse, dout, dq, dk, dv, B, H, N, d, scale, causal, stream):
     """attn_bwd with its scratch in a fixed array inside the library, for callers
     that cannot allocate device memory (include/attn_b200.h)."""
@@ -167,7 +177,10 @@ def use_library(path):
 
 
 def attn_get_device_status(stream):
-    return load().attn_get_device_status(stream)
+    st = load().attn_get_device_status(stream)
+    if st != ATTN_OK and _W4_WORKSPACES:
+        _reset_w4_workspaces()
+    return st
 
 
 def attn_status_string(status):
@@ -448,9 +461,42 @@ def backward(q, k, v, o, lse, dout, causal=False, scale=None, dq=None, dk=None, 
     return dq, dk, dv
 
 
-def w4a16_matmul(x, qweight, scales, zeros, out=None, stream=None, check=False):
+# split-K workspaces of w4a16_matmul, one per (device, stream): zeroed when
+# allocated; every call leaves the tickets zero again
+_W4_WORKSPACES = {}
+
+
+def _reset_w4_workspaces():
+    """After a device status other than ATTN_OK a split-K call may have left
+    tickets set: wait for the device and zero every cached workspace."""
+    import torch
+    torch.cuda.synchronize()
+    for t in _W4_WORKSPACES.values():
+        t.zero_()
+    torch.cuda.synchronize()
+
+
+def _w4_workspace(device, stream_ptr, nbytes):
+    import torch
+    key = (device.index, stream_ptr)
+    ws = _W4_WORKSPACES.get(key)
+    if ws is None or ws.numel() < nbytes:
+        if ws is not None:
+            torch.cuda.synchronize(device)        # the old one may still be read by a launch
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        torch.cuda.current_stream(device).synchronize()   # zeroed before any stream uses it
+        _W4_WORKSPACES[key] = ws
+    return ws
+
+
+def w4a16_matmul(x, qweight, scales, zeros, out=None, stream=None, check=False, split_k=True, workspace=None):
     """Y = X W for fp16 X [M, K] and W given as packed int4 (int32 [K/8, N]), fp16
-    scales [K/128, N] and uint8 zero points [K/128, N] (include/w4a16_b200.h)."""
+    scales [K/128, N] and uint8 zero points [K/128, N] (include/w4a16_b200.h).
+
+    split_k=True (default) runs w4a16_gemm_splitk, which balances the K slices over
+    every SM; its workspace is `workspace` (a zeroed uint8 CUDA tensor of at least
+    w4a16_gemm_splitk_workspace_bytes(M, N, K) bytes) or one cached per device and
+    stream. split_k=False runs w4a16_gemm (one CTA per 128 output columns)."""
     import torch
     if x.dim() != 2:
         raise ValueError("x must be [M, K]")
@@ -464,9 +510,23 @@ def w4a16_matmul(x, qweight, scales, zeros, out=None, stream=None, check=False):
         out = torch.empty((M, N), dtype=torch.float16, device=x.device)
     _expect(out, "out", (M, N), torch.float16, x.device)
     sp = _stream_ptr(x, stream)
-    _check(w4a16_gemm(x.data_ptr(), qweight.data_ptr(), scales.data_ptr(), zeros.data_ptr(), out.data_ptr(),
-                      M, N, K, sp), "w4a16_gemm")
-    _check_device(check, sp, "w4a16_gemm")
+    if not split_k:
+        _check(w4a16_gemm(x.data_ptr(), qweight.data_ptr(), scales.data_ptr(), zeros.data_ptr(), out.data_ptr(),
+                          M, N, K, sp), "w4a16_gemm")
+        _check_device(check, sp, "w4a16_gemm")
+        return out
+    need = w4a16_gemm_splitk_workspace_bytes(M, N, K)
+    if need == 0:
+        raise AttnError(ATTN_ERR_UNSUPPORTED, "w4a16_gemm_splitk_workspace_bytes")
+    if workspace is None:
+        workspace = _w4_workspace(x.device, sp, need)
+    elif workspace.device != x.device or not workspace.is_contiguous() or \
+            workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace must be a contiguous tensor of at least {need} bytes on {x.device}")
+    _check(w4a16_gemm_splitk(x.data_ptr(), qweight.data_ptr(), scales.data_ptr(), zeros.data_ptr(),
+                             out.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             M, N, K, sp), "w4a16_gemm_splitk")
+    _check_device(check, sp, "w4a16_gemm_splitk")
     return out
 
 

@@ -611,8 +611,21 @@ attn_status attn_bwd(const void* q, const void* k, const void* v, const void* o,
   return launch_bwd<64>(q, k, v, o, lse, dout, dq, dk, dv, dd, B * H, N, scale, causal, st);
 }
 
-attn_status w4a16_gemm(const void* x, const void* qweight, const void* scales, const void* zeros, void* y, int M,
-                       int N, int K, void* stream) {
+namespace {
+
+constexpr int kW4MaxCtas = 296;      // two per SM of a B200: the most a split-K launch uses
+constexpr int kW4MinSlices = 8;      // a split-K run covers at least this many 128-deep slices
+
+// Split-K CTA cap for U units, before the device's SM count is applied.
+int w4_cta_cap(long long units) {
+  const long long c = units / kW4MinSlices;
+  return static_cast<int>(c < 1 ? 1 : (c > kW4MaxCtas ? kW4MaxCtas : c));
+}
+
+size_t w4_tickets_bytes(int N) { return static_cast<size_t>((16ll * (N / 128) + 255) / 256 * 256); }
+
+attn_status w4_check(const void* x, const void* qweight, const void* scales, const void* zeros, const void* y, int M,
+                     int N, int K) {
   using C = attn::W4Cfg;
   if (x == nullptr || qweight == nullptr || scales == nullptr || zeros == nullptr || y == nullptr)
     return ATTN_ERR_INVALID_ARG;
@@ -621,6 +634,13 @@ attn_status w4a16_gemm(const void* x, const void* qweight, const void* scales, c
   if (!aligned16(x) || !aligned16(qweight) || !aligned16(scales) || !aligned16(zeros) || !aligned16(y))
     return ATTN_ERR_MISALIGNED;
   if (static_cast<long long>(K) * N >= (1ll << 40)) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
+// One launch of w4a16_gemm_sm100 over `ctas` CTAs (ctas = N / 128: a tile each).
+attn_status launch_w4(const void* x, const void* qweight, const void* scales, const void* zeros, void* y, void* ws,
+                      int M, int N, int K, int ctas, cudaStream_t stream) {
+  using C = attn::W4Cfg;
   const int mpad = (M + 15) / 16 * 16;
   CUtensorMap tx, tw, ts, tz;
   if (!encode_matrix_map(&tx, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, K, M, 64, mpad, true) ||
@@ -636,14 +656,52 @@ attn_status w4a16_gemm(const void* x, const void* qweight, const void* scales, c
   p.N = N;
   p.K = K;
   p.mpad = mpad;
+  p.ctas = ctas;
+  p.units = static_cast<long long>(N / C::BN) * (K / C::GROUP);
   p.y = static_cast<__half*>(y);
+  p.tickets = ws == nullptr ? nullptr : static_cast<uint32_t*>(ws);
+  p.part = ws == nullptr ? nullptr
+                         : reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + w4_tickets_bytes(N));
   p.timeout_cycles = kWaitLimitCycles;
-  attn::w4a16_gemm_sm100<<<N / C::BN, C::THREADS, smem, static_cast<cudaStream_t>(stream)>>>(tx, tw, ts, tz, p);
+  attn::w4a16_gemm_sm100<<<ctas, C::THREADS, smem, stream>>>(tx, tw, ts, tz, p);
   if (cudaGetLastError() != cudaSuccess) {
     forget_smem(9);
     return ATTN_ERR_CUDA;
   }
   return ATTN_OK;
+}
+
+}  // namespace
+
+attn_status w4a16_gemm(const void* x, const void* qweight, const void* scales, const void* zeros, void* y, int M,
+                       int N, int K, void* stream) {
+  if (attn_status s = w4_check(x, qweight, scales, zeros, y, M, N, K); s != ATTN_OK) return s;
+  return launch_w4(x, qweight, scales, zeros, y, nullptr, M, N, K, N / attn::W4Cfg::BN,
+                   static_cast<cudaStream_t>(stream));
+}
+
+size_t w4a16_gemm_splitk_workspace_bytes(int M, int N, int K) {
+  using C = attn::W4Cfg;
+  if (M < 1 || N < 1 || K < 1 || M > C::MAX_M || N % C::BN != 0 || K % C::GROUP != 0) return 0;
+  if (static_cast<long long>(K) * N >= (1ll << 40)) return 0;
+  const long long mpad = (M + 15) / 16 * 16;
+  const int cap = w4_cta_cap(static_cast<long long>(N / C::BN) * (K / C::GROUP));
+  return w4_tickets_bytes(N) + static_cast<size_t>(2ll * cap * mpad * C::BN * 4);
+}
+
+attn_status w4a16_gemm_splitk(const void* x, const void* qweight, const void* scales, const void* zeros, void* y,
+                              void* workspace, size_t workspace_bytes, int M, int N, int K, void* stream) {
+  using C = attn::W4Cfg;
+  if (attn_status s = w4_check(x, qweight, scales, zeros, y, M, N, K); s != ATTN_OK) return s;
+  if (workspace == nullptr || workspace_bytes < w4a16_gemm_splitk_workspace_bytes(M, N, K))
+    return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
+  const int sms = sm_count();
+  if (sms <= 0) return ATTN_ERR_CUDA;
+  const long long units = static_cast<long long>(N / C::BN) * (K / C::GROUP);
+  const int cap = w4_cta_cap(units);
+  const int ctas = 2 * sms < cap ? 2 * sms : cap;
+  return launch_w4(x, qweight, scales, zeros, y, workspace, M, N, K, ctas, static_cast<cudaStream_t>(stream));
 }
 
 attn_status attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,

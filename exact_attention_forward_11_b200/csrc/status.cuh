@@ -39,6 +39,7 @@ enum DebugSite : uint32_t {
   kSiteW4Out = 9,          // output column store, W4A16 GEMM
   kSiteTmaCoord = 10,      // TMA coordinate (x not a multiple of 16 elements, a negative store
                            // coordinate, or a unit outside the launch)
+  kSiteW4Split = 11,       // partial slot or ticket index, split-K W4A16 GEMM
 };
 
 __device__ uint32_t g_status;

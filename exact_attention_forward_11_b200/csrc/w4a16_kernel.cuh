@@ -11,8 +11,16 @@
 //   PERM = 0 2 4 6 1 3 5 7), fp32 accumulation, Y rounded to fp16.
 //
 // Decode-sized M (1..128 tokens) makes the GEMM HBM-bound on the weights (half a
-// byte per weight), so the layout is chosen for a stream: one CTA per 128 output
-// columns walks K in 128-deep slices. The MMA is issued with the operands swapped
+// byte per weight), so the layout is chosen for a stream: a CTA walks K in
+// 128-deep slices of 128 output columns. The work is the list of (column tile,
+// slice) units, tile-major; CTA c of C takes units [c U / C, (c+1) U / C). With
+// C = the number of tiles every CTA owns one whole tile. With C = two per SM
+// (balanced split-K) a CTA's run may start or end inside a tile: the part of a
+// tile it covers is a segment, written as an fp32 partial to a caller workspace
+// slot (2c for the run's first tile, 2c+1 for its last); the warp that takes the
+// last ticket of its tile's 32-column quarter adds the tile's partials in CTA
+// order (so the sum does not depend on which CTA finishes last), writes Y and
+// resets the ticket. The MMA is issued with the operands swapped
 // (D[128 columns n][M tokens] = W^T X^T) so that M = 128 is the weight side and
 // the token count only sets the MMA's N (padded to a multiple of 16). The
 // dequantised weights go straight from registers into tensor memory (one thread
@@ -23,9 +31,11 @@
 // slice of each K slice into a ring of up to 8 stages), warp 1 MMA issuer (owns
 // TMEM), warps 2-3 idle, warps 4-11 dequantise (thread t of quarter q: column
 // n0 + 32 q + t; warps 4-7 take the first 8 words of a slice, 8-11 the last 8)
-// and warps 4-7 write Y. Two CTAs fit on an SM (85 registers per thread).
+// and warps 4-7 write each segment's Y or partial. Two CTAs fit on an SM.
 // TMEM: three (two for M > 64) 64-column A buffers (a 128-deep slice of fp16
-// pairs each) and the MPAD-column fp32 accumulator. Every wait is bounded (Waiter).
+// pairs each) and the MPAD-column fp32 accumulator, which the MMA reuses for the
+// next segment once warps 4-7 have read it. Every wait is bounded (Waiter); the
+// tickets are atomics, never waited on.
 #pragma once
 
 #include <cstdint>
@@ -74,7 +84,7 @@ struct W4Cfg {
   }
   __host__ __device__ static constexpr int bar_offset(int mpad) { return nst(mpad) * stage_bytes(mpad); }
   __host__ __device__ static constexpr int smem_bytes(int mpad) {
-    return bar_offset(mpad) + (2 * MAX_NST + 2 * MAX_NA + 2) * 8 + 16 + 1024;
+    return bar_offset(mpad) + (2 * MAX_NST + 2 * MAX_NA + 3) * 8 + 32 + 1024;
   }
   // the largest smem_bytes over every M (the kernel attribute must cover all)
   __host__ static constexpr int max_smem_bytes() {
@@ -87,9 +97,21 @@ struct W4Cfg {
 struct W4Params {
   int M, N, K;
   int mpad;                  // M rounded up to a multiple of 16
+  int ctas;                  // C: CTAs of the launch (the grid)
+  long long units;           // U = (N / 128) * (K / 128)
   __half* y;                 // [M, N]
+  float* part;               // [2 C][mpad][128] fp32 segment partials (split-K only)
+  uint32_t* tickets;         // [4 N / 128] per tile quarter, zero between launches (split-K only)
   uint64_t timeout_cycles;
 };
+
+// First unit of CTA c, and the CTA whose run holds unit u.
+__host__ __device__ __forceinline__ long long w4_unit0(int c, long long U, int C) {
+  return static_cast<long long>(c) * U / C;
+}
+__host__ __device__ __forceinline__ int w4_cta_of(long long u, long long U, int C) {
+  return static_cast<int>(((u + 1) * C - 1) / U);
+}
 
 __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     w4a16_gemm_sm100(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
@@ -110,14 +132,16 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
   const uint32_t T_D = C::t_d(mpad);
   uint64_t* a_full = empty + C::MAX_NST;     // NA: 4 dequant warps
   uint64_t* a_empty = a_full + C::MAX_NA;    // NA: MMA commit
-  uint64_t* done = a_empty + C::MAX_NA;      // 1
-  uint64_t* drain_bar = done + 1;            // 1
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::MAX_NST + 2 * C::MAX_NA + 2);
+  uint64_t* seg_done = a_empty + C::MAX_NA;  // 1: MMA commit at each segment's end
+  uint64_t* d_free = seg_done + 1;           // 1: warps 4-7 have read the accumulator
+  uint64_t* drain_bar = d_free + 1;          // 1
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::MAX_NST + 2 * C::MAX_NA + 3);
   uint32_t* abort_word = tmem_slot + 1;
+  int* run_info = reinterpret_cast<int*>(tmem_slot + 2);   // [units in the run, first tile, first slice]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * C::BN;
-  const int G = p.K / C::GROUP;              // slices
+  const int G = p.K / C::GROUP;              // slices per tile
+  const long long U = p.units;
 
   auto x_at = [&](int s) { return smem + s * SB; };
   auto w_at = [&](int s) { return reinterpret_cast<const uint32_t*>(smem + s * SB + 2 * XC); };
@@ -133,9 +157,15 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
       mbar_init(a_full + b, 4 * C::SPLIT);
       mbar_init(a_empty + b, 1);
     }
-    mbar_init(done, 1);
+    mbar_init(seg_done, 1);
+    mbar_init(d_free, 4);
     mbar_init(drain_bar, 1);
     *abort_word = 0u;
+    // the run, computed once here (64-bit divisions) and read back from shared memory
+    const long long u0 = w4_unit0(blockIdx.x, U, p.ctas);
+    run_info[0] = static_cast<int>(w4_unit0(blockIdx.x + 1, U, p.ctas) - u0);
+    run_info[1] = static_cast<int>(u0 / G);
+    run_info[2] = static_cast<int>(u0 - static_cast<long long>(run_info[1]) * G);
     fence_barrier_init();
     fence_proxy_async_shared();
   }
@@ -147,10 +177,14 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // this CTA's run: n_units units from slice g0 of tile tile0
+  const int n_units = run_info[0], tile0 = run_info[1], g0 = run_info[2];
   const Waiter waiter{abort_word, p.timeout_cycles};
   auto wait_all = [&](uint64_t* bar, uint32_t parity) { return __all_sync(0xffffffffu, waiter.wait(bar, parity)); };
   bool ok = true;
 
+  // Every role walks the run as segments (outer loop: one tile each) of slices
+  // [gs, ge) (inner loop); i counts units across the run for the ring phases.
   if (warp == 0) {
     // ======================= producer =======================
     if (elect_one()) {
@@ -163,24 +197,27 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     const uint64_t pol_w = l2_policy_evict_first();   // weights are read once
     const uint64_t pol_x = l2_policy_evict_last();    // X is read by every CTA
     const uint32_t bytes = static_cast<uint32_t>(2 * XC + C::WQ_BYTES + C::S_BYTES + C::Z_BYTES);
-    int g = 0;
-    for (; g < G; ++g) {
-      const int s = g % NST;
-      if (g >= NST && !(ok = wait_all(empty + s, ((g / NST) - 1) & 1))) break;
-      if (elect_one()) {
-        mbar_arrive_expect_tx(full + s, bytes);
-        tma_load_3d(x_at(s), &tm_x, full + s, g * C::GROUP, 0, 0, pol_x);
-        tma_load_3d(x_at(s) + XC, &tm_x, full + s, g * C::GROUP + 64, 0, 0, pol_x);
-        tma_load_3d(const_cast<uint32_t*>(w_at(s)), &tm_w, full + s, n0, g * 16, 0, pol_w);
-        tma_load_3d(const_cast<__half*>(s_at(s)), &tm_s, full + s, n0, g, 0, pol_w);
-        tma_load_3d(z_at(s), &tm_z, full + s, n0, g, 0, pol_w);
+    int i = 0, s = 0, r = 0;                 // unit, its ring stage, and the ring round
+    for (int tile = tile0, gs = g0; ok && i < n_units; ++tile, gs = 0) {
+      const int ge = min(G, gs + (n_units - i));
+      const int n0 = tile * C::BN;
+      for (int g = gs; g < ge; ++g, ++i, s = (s == NST - 1 ? 0 : s + 1), r += (s == 0)) {
+        if (r > 0 && !(ok = wait_all(empty + s, (r - 1) & 1))) break;
+        if (elect_one()) {
+          mbar_arrive_expect_tx(full + s, bytes);
+          tma_load_3d(x_at(s), &tm_x, full + s, g * C::GROUP, 0, 0, pol_x);
+          tma_load_3d(x_at(s) + XC, &tm_x, full + s, g * C::GROUP + 64, 0, 0, pol_x);
+          tma_load_3d(const_cast<uint32_t*>(w_at(s)), &tm_w, full + s, n0, g * 16, 0, pol_w);
+          tma_load_3d(const_cast<__half*>(s_at(s)), &tm_s, full + s, n0, g, 0, pol_w);
+          tma_load_3d(z_at(s), &tm_z, full + s, n0, g, 0, pol_w);
+        }
+        __syncwarp();
       }
-      __syncwarp();
     }
     if (!ok) {
       if (lane == 0) record_timeout();
       const uint64_t t0 = sm_clock();
-      for (int j = (g > NST ? g - NST : 0); j < g; ++j)
+      for (int j = (i > NST ? i - NST : 0); j < i; ++j)
         while (!mbar_try_wait(full + (j % NST), (j / NST) & 1) && sm_clock() - t0 < p.timeout_cycles) {
         }
     }
@@ -190,22 +227,28 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     const uint32_t idesc = instr_desc(0u /* f16 */, 128, static_cast<uint32_t>(mpad), 0, 0);
     constexpr uint32_t hi = smem_desc_hi(1024);
     const uint32_t x_lo = smem_desc_lo(smem_addr(smem), 16);
-    for (int g = 0; g < G; ++g) {
-      const int s = g % NST, b = g % NA;
-      if (!(ok = wait_all(full + s, (g / NST) & 1))) break;
-      if (!(ok = wait_all(a_full + b, (g / NA) & 1))) break;
-      tc_fence_after();
-      const uint32_t xa = x_lo + ((s * SB) >> 4);
+    int i = 0, s = 0, r = 0, b = 0, ra = 0;  // unit; ring stage and round; A buffer and its round
+    for (int seg = 0, gs = g0; ok && i < n_units; ++seg, gs = 0) {
+      const int ge = min(G, gs + (n_units - i));
+      // the accumulator is reused: the previous segment must have been read
+      if (seg > 0 && !(ok = wait_all(d_free, (seg - 1) & 1))) break;
+      for (int g = gs; g < ge; ++g, ++i, s = (s == NST - 1 ? 0 : s + 1), r += (s == 0),
+               b = (b == NA - 1 ? 0 : b + 1), ra += (b == 0)) {
+        if (!(ok = wait_all(full + s, r & 1))) break;
+        if (!(ok = wait_all(a_full + b, ra & 1))) break;
+        tc_fence_after();
+        const uint32_t xa = x_lo + ((s * SB) >> 4);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = ((kk >> 2) * XC + (kk & 3) * 32) >> 4;
-        mma_f16_ts(tmem_base + T_D, tmem_base + C::T_A + 64 * b + 8 * kk, smem_desc(xa + off, hi), idesc,
-                   (g > 0 || kk > 0) ? 1u : 0u, leader);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = ((kk >> 2) * XC + (kk & 3) * 32) >> 4;
+          mma_f16_ts(tmem_base + T_D, tmem_base + C::T_A + 64 * b + 8 * kk, smem_desc(xa + off, hi), idesc,
+                     (g > gs || kk > 0) ? 1u : 0u, leader);
+        }
+        mma_commit(empty + s, leader);
+        mma_commit(a_empty + b, leader);
       }
-      mma_commit(empty + s, leader);
-      mma_commit(a_empty + b, leader);
+      if (ok) mma_commit(seg_done, leader);
     }
-    if (ok) mma_commit(done, leader);
     if (!ok && lane == 0) record_timeout();
     mma_commit(drain_bar, leader);
     const uint64_t t0 = sm_clock();
@@ -213,62 +256,108 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ======================= dequantise, then Y =======================
+    // ======================= dequantise; Y or partial at each segment's end =======================
     const int wq = warp & 3;                         // TMEM lane quarter
     const int h = (warp - 4) >> 2;                   // which words of the slice (SPLIT 2)
     const int t = wq * 32 + lane;                    // output column n0 + t, TMEM lane t
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    for (int g = 0; g < G; ++g) {
-      const int s = g % NST, b = g % NA;
-      if (!(ok = wait_all(full + s, (g / NST) & 1))) break;
-      if (g >= NA && !(ok = wait_all(a_empty + b, ((g / NA) - 1) & 1))) break;
-      const __half2 ss = __half2half2(s_at(s)[t]);
-      // 1024 + z as fp16: the unpacked words below hold 1024 + q (exponent bits
-      // 0x6400 with q in the low mantissa bits), so one subtraction gives q - z exactly
-      const __half zh = __ushort_as_half(static_cast<unsigned short>(0x6400u | z_at(s)[t]));
-      const __half2 zz = __half2half2(zh);
-      const uint32_t* wrow = w_at(s);
-      uint32_t pk[4 * C::WORDS];
+    int i = 0, s = 0, r = 0, b = 0, ra = 0;  // unit; ring stage and round; A buffer and its round
+    for (int seg = 0, tile = tile0, gs = g0; ok && i < n_units; ++seg, ++tile, gs = 0) {
+      const int ge = min(G, gs + (n_units - i));
+      for (int g = gs; g < ge; ++g, ++i, s = (s == NST - 1 ? 0 : s + 1), r += (s == 0),
+               b = (b == NA - 1 ? 0 : b + 1), ra += (b == 0)) {
+        if (!(ok = wait_all(full + s, r & 1))) break;
+        if (ra > 0 && !(ok = wait_all(a_empty + b, (ra - 1) & 1))) break;
+        const __half2 ss = __half2half2(s_at(s)[t]);
+        // 1024 + z as fp16: the unpacked words below hold 1024 + q (exponent bits
+        // 0x6400 with q in the low mantissa bits), so one subtraction gives q - z exactly
+        const __half zh = __ushort_as_half(static_cast<unsigned short>(0x6400u | z_at(s)[t]));
+        const __half2 zz = __half2half2(zh);
+        const uint32_t* wrow = w_at(s);
+        uint32_t pk[4 * C::WORDS];
 #pragma unroll
-      for (int i = 0; i < C::WORDS; ++i) {
-        const uint32_t word = wrow[(C::WORDS * h + i) * C::BN + t];
+        for (int k = 0; k < C::WORDS; ++k) {
+          const uint32_t word = wrow[(C::WORDS * h + k) * C::BN + t];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          // bits 4j..4j+3 (weight 8i+2j) into the low half, bits 16+4j.. (8i+2j+1) into the high half
-          const uint32_t v = ((word >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
-          const __half2 h = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v), zz), ss);
-          pk[4 * i + j] = *reinterpret_cast<const uint32_t*>(&h);
+          for (int j = 0; j < 4; ++j) {
+            // bits 4j..4j+3 (weight 8k+2j) into the low half, bits 16+4j.. (8k+2j+1) into the high half
+            const uint32_t v = ((word >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+            const __half2 hv = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v), zz), ss);
+            pk[4 * k + j] = *reinterpret_cast<const uint32_t*>(&hv);
+          }
         }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty + s);         // this warp's words, scale and zero are read
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + s);       // this warp's words, scale and zero are read
 #pragma unroll
-      for (int q = 0; q < C::WORDS / 8; ++q)
-        tmem_st32(tmem_base + lane_off + C::T_A + 64 * b + 4 * C::WORDS * h + 32 * q, pk + 32 * q);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(a_full + b);
-    }
-    // Y: the first warpgroup reads the accumulator and writes the tile
-    if (ok && h == 0) ok = wait_all(done, 0);
-    if (!ok) {
-      if (lane == 0) record_timeout();
-    } else if (h == 0) {
+        for (int q = 0; q < C::WORDS / 8; ++q)
+          tmem_st32(tmem_base + lane_off + C::T_A + 64 * b + 4 * C::WORDS * h + 32 * q, pk + 32 * q);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(a_full + b);
+      }
+      if (!ok) break;
+      if (h != 0) continue;
+      // ---- segment end (warps 4-7): read the accumulator, then Y or a partial ----
+      if (!(ok = wait_all(seg_done, seg & 1))) break;
       tc_fence_after();
-      __half* ycol = p.y + n0 + t;
+      const long long tu0 = static_cast<long long>(tile) * G;
+      const int c_lo = w4_cta_of(tu0, U, p.ctas), c_hi = w4_cta_of(tu0 + G - 1, U, p.ctas);
+      const int n0 = tile * C::BN;
+      const bool whole = c_lo == c_hi;
       const bool col_ok = dbg_ok(n0 + t < p.N, kSiteW4Out, static_cast<unsigned>(n0 + t));
+      const int slot = 2 * static_cast<int>(blockIdx.x) + (tile == tile0 ? 0 : 1);
+      const bool part_ok = whole || dbg_ok(slot < 2 * p.ctas && tile < p.N / C::BN, kSiteW4Split,
+                                           static_cast<unsigned long long>(slot));
+      float* mine = whole ? nullptr : p.part + static_cast<size_t>(slot) * mpad * C::BN;
       for (int c0 = 0; c0 < mpad; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem_base + lane_off + T_D + c0, v);
         tmem_ld_wait<16>(v);
+        if (c0 + 16 >= mpad) {                       // the accumulator is free for the next segment
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(d_free);
+        }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int m = c0 + i;
-          if (m < p.M && col_ok) ycol[static_cast<size_t>(m) * p.N] = __float2half_rn(__uint_as_float(v[i]));
+        for (int k = 0; k < 16; ++k) {
+          const int m = c0 + k;
+          if (whole) {
+            if (m < p.M && col_ok) p.y[static_cast<size_t>(m) * p.N + n0 + t] = __float2half_rn(__uint_as_float(v[k]));
+          } else if (part_ok) {
+            __stcg(mine + static_cast<size_t>(m) * C::BN + t, __uint_as_float(v[k]));
+          }
         }
       }
+      if (whole || !part_ok) continue;
+      // publish this segment's quarter; the last of the tile's segments sums them in CTA order
+      __threadfence();
+      __syncwarp();
+      uint32_t prev = 0;
+      uint32_t* ticket = p.tickets + 4 * tile + wq;
+      if (lane == 0) prev = atomicAdd(ticket, 1u);
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+      if (prev != static_cast<uint32_t>(c_hi - c_lo)) continue;
+      __threadfence();
+      for (int c0 = 0; c0 < p.M; c0 += 8) {          // 8 rows at a time, partials added in CTA order
+        float acc[8];
+        for (int c = c_lo; c <= c_hi; ++c) {
+          const int ht = static_cast<int>(w4_unit0(c, U, p.ctas) / G);
+          const float* src = p.part + (static_cast<size_t>(2 * c + (ht == tile ? 0 : 1)) * mpad + c0) * C::BN + t;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const float val = __ldcg(src + k * C::BN);
+            acc[k] = c == c_lo ? val : acc[k] + val;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          if (c0 + k < p.M && col_ok) p.y[static_cast<size_t>(c0 + k) * p.N + n0 + t] = __float2half_rn(acc[k]);
+      }
+      __syncwarp();
+      if (lane == 0) *ticket = 0u;                   // ready for the next launch
     }
+    if (!ok && lane == 0) record_timeout();
   }
 
   tc_fence_before();

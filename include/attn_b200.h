@@ -261,7 +261,8 @@ ATTN_API attn_status attn_get_device_status(void* stream);
  * none). Sites: 1 O / LSE row (two-Q-tile forward), 2 O / LSE row (one-Q-tile
  * forward), 3 MXFP8 scale-byte row load, 4 dK / dV row, 5 LSE / D_i load (dK dV
  * kernel), 6 dQ row and its LSE / D_i load, 7 FP8 tile scale, 8 MXFP8 block,
- * 9 W4A16 output column, 10 TMA coordinate or work unit. `site` and `index`
+ * 9 W4A16 output column, 10 TMA coordinate or work unit, 11 split-K W4A16
+ * partial slot (index: the slot). `site` and `index`
  * are host pointers. Returns ATTN_OK, ATTN_ERR_INVALID_ARG for a null pointer,
  * or ATTN_ERR_CUDA. In a release build the site is always 0.
  */

@@ -148,6 +148,40 @@ def test_w4a16_argument_validation(lib):
     assert call(4, FAKE + 2) == lib.ATTN_ERR_MISALIGNED
 
 
+def test_w4a16_splitk_workspace_and_validation(lib):
+    """Workspace size of the split-K W4A16 call: the tickets (16 bytes per 128
+    columns, rounded up to 256) plus two fp32 slots of mpad x 128 values for each
+    of at most 296 CTAs, one CTA per 8 slices for small problems; argument
+    errors come back before any CUDA call."""
+    wsb = lib.w4a16_gemm_splitk_workspace_bytes
+    # decode MLP shape: 224 tiles x 64 slices -> 296 CTAs
+    assert wsb(16, 28672, 8192) == 3584 + 2 * 296 * 16 * 128 * 4
+    assert wsb(1, 28672, 8192) == wsb(16, 28672, 8192)            # M padded to 16
+    assert wsb(17, 28672, 8192) == 3584 + 2 * 296 * 32 * 128 * 4
+    # 8 tiles x 32 slices = 256 units -> 32 CTAs
+    assert wsb(16, 1024, 4096) == 256 + 2 * 32 * 16 * 128 * 4
+    # one unit -> one CTA
+    assert wsb(128, 128, 128) == 256 + 2 * 1 * 128 * 128 * 4
+    for bad in ((0, 128, 128), (129, 128, 128), (16, 200, 128), (16, 128, 100), (16, -128, 128)):
+        assert wsb(*bad) == 0
+    f = lib.w4a16_gemm_splitk
+    need = wsb(16, 256, 512)
+    ok = [FAKE] * 6 + [need, 16, 256, 512, None]
+
+    def call(i=None, val=None):
+        a = list(ok)
+        if i is not None:
+            a[i] = val
+        return f(*a)
+    assert call(5, None) == lib.ATTN_ERR_INVALID_ARG           # no workspace
+    assert call(6, need - 16) == lib.ATTN_ERR_INVALID_ARG      # workspace too small
+    assert call(5, FAKE + 8) == lib.ATTN_ERR_MISALIGNED
+    assert call(1, None) == lib.ATTN_ERR_INVALID_ARG
+    assert call(7, 129) == lib.ATTN_ERR_UNSUPPORTED
+    assert call(8, 200) == lib.ATTN_ERR_UNSUPPORTED
+    assert call(4, FAKE + 2) == lib.ATTN_ERR_MISALIGNED
+
+
 def test_debug_build_exports_the_same_boundary(lib):
     """The debug build (-DATTN_DEBUG) builds, exports every declared symbol, says
     it is the debug build, and validates arguments on the host like the release
