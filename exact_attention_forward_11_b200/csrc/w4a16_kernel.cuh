@@ -268,22 +268,48 @@ __global__ void __launch_bounds__(W4Cfg::THREADS, 2)
                b = (b == NA - 1 ? 0 : b + 1), ra += (b == 0)) {
         if (!(ok = wait_all(full + s, r & 1))) break;
         if (ra > 0 && !(ok = wait_all(a_empty + b, (ra - 1) & 1))) break;
-        const __half2 ss = __half2half2(s_at(s)[t]);
+        const __half sh = s_at(s)[t];
+        const uint32_t zb = z_at(s)[t];
+        const __half2 ss = __half2half2(sh);
         // 1024 + z as fp16: the unpacked words below hold 1024 + q (exponent bits
         // 0x6400 with q in the low mantissa bits), so one subtraction gives q - z exactly
-        const __half zh = __ushort_as_half(static_cast<unsigned short>(0x6400u | z_at(s)[t]));
-        const __half2 zz = __half2half2(zh);
+        const __half2 zz = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6400u | zb)));
+        // Nibbles masked in place one position higher (bits 4..7 of a half) read as
+        // 1024 + 16 q: less 1024 + 16 z that is 16 (q - z), exact, and times s / 16 it is
+        // the same real product (q - z) s, rounded once: the same fp16 value, one shift
+        // fewer per nibble pair. Taken when s / 16 is exact (s * 2^-4 times 16 gives s
+        // back) for every lane of the warp; otherwise every pair goes the shifting way.
+        const __half s16 = __hmul(sh, __ushort_as_half(static_cast<unsigned short>(0x2C00u)));   // 2^-4
+        const bool exact16 = __heq(__hmul(s16, __ushort_as_half(static_cast<unsigned short>(0x4C00u))), sh);
         const uint32_t* wrow = w_at(s);
         uint32_t pk[4 * C::WORDS];
+        if (__all_sync(0xffffffffu, exact16)) {
+          const __half2 ss16 = __half2half2(s16);
+          const __half2 zz16 = __half2half2(__ushort_as_half(static_cast<unsigned short>(0x6400u | (zb << 4))));
 #pragma unroll
-        for (int k = 0; k < C::WORDS; ++k) {
-          const uint32_t word = wrow[(C::WORDS * h + k) * C::BN + t];
+          for (int k = 0; k < C::WORDS; ++k) {
+            const uint32_t word = wrow[(C::WORDS * h + k) * C::BN + t];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            // bits 4j..4j+3 (weight 8k+2j) into the low half, bits 16+4j.. (8k+2j+1) into the high half
-            const uint32_t v = ((word >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
-            const __half2 hv = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v), zz), ss);
-            pk[4 * k + j] = *reinterpret_cast<const uint32_t*>(&hv);
+            for (int j = 0; j < 4; ++j) {
+              // pairs 2j, 2j+1: bits 4j..4j+3 and 16+4j..; odd j stays 4 bits up
+              const uint32_t src = j < 2 ? word : word >> 8;
+              const uint32_t v = (src & ((j & 1) ? 0x00F000F0u : 0x000F000Fu)) | 0x64006400u;
+              const __half2 hv = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v), (j & 1) ? zz16 : zz),
+                                         (j & 1) ? ss16 : ss);
+              pk[4 * k + j] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int k = 0; k < C::WORDS; ++k) {
+            const uint32_t word = wrow[(C::WORDS * h + k) * C::BN + t];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              // bits 4j..4j+3 (weight 8k+2j) into the low half, bits 16+4j.. (8k+2j+1) into the high half
+              const uint32_t v = ((word >> (4 * j)) & 0x000F000Fu) | 0x64006400u;
+              const __half2 hv = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&v), zz), ss);
+              pk[4 * k + j] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
           }
         }
         __syncwarp();

@@ -126,6 +126,43 @@ def test_w4a16_dequantisation_bit_exact(cuda_lib):
     np.testing.assert_array_equal(y, w[ks].astype(np.float32))
 
 
+def _scales(kind, shape, seed):
+    """fp16 scales of one regime: typical ([0.005, 0.02)), tiny (2^-20 .. 2^-10, where
+    s / 16 is mostly not an fp16 value), mixed (typical and tiny columns alternate, so
+    every warp holds both), powers (2^-8 .. 2^-24: s / 16 exact down to 2^-20 only)."""
+    gen = torch.Generator().manual_seed(seed)
+    typical = (torch.rand(shape, generator=gen) * 0.015 + 0.005).to(torch.float16)
+    tiny = torch.exp2(-10.0 - 10.0 * torch.rand(shape, generator=gen)).to(torch.float16)
+    if kind == "typical":
+        return typical
+    if kind == "tiny":
+        return tiny
+    if kind == "mixed":
+        out = typical.clone()
+        out[:, 1::2] = tiny[:, 1::2]
+        return out
+    e = torch.randint(8, 25, shape, generator=gen).to(torch.float32)
+    return torch.exp2(-e).to(torch.float16)
+
+
+@pytest.mark.parametrize("split_k", [True, False], ids=["splitk", "tile_per_cta"])
+@pytest.mark.parametrize("kind", ["typical", "tiny", "mixed", "powers"])
+def test_w4a16_dequantisation_bit_exact_scale_regimes(cuda_lib, kind, split_k):
+    """The kernel unpacks odd nibble pairs without a shift (16 (q - z) times s / 16)
+    when s / 16 is exact for a whole warp and takes the shifting form otherwise;
+    both must give fp16((q - z) s) bit for bit, for every scale regime."""
+    K, N = 256, 384
+    _, qw, _, z = workloads.make_w4a16(1, N, K, seed=11)
+    s = _scales(kind, (K // 128, N), seed=12)
+    ks = list(range(0, 16)) + [127, 128, 135, 200, 255]
+    x = torch.zeros((len(ks), K), dtype=torch.float16)
+    for m, k in enumerate(ks):
+        x[m, k] = 1.0
+    y = run(cuda_lib, x, qw, s, z, split_k=split_k)
+    w = dequantize_weights(qw.numpy(), s.numpy(), z.numpy())
+    np.testing.assert_array_equal(y, w[ks].astype(np.float32))
+
+
 @pytest.mark.parametrize("split_k", [True, False], ids=["splitk", "tile_per_cta"])
 def test_w4a16_workload_parity(cuda_lib, split_k):
     """The decode workload at full size (split-K is the launch the benchmark
