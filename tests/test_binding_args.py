@@ -48,3 +48,27 @@ def test_every_argument_is_checked(cuda_lib):
         cuda_lib.forward_fp8(c, c.cpu(), c, s, s, s)
     torch.cuda.synchronize()
     assert cuda_lib.attn_get_device_status(None) == cuda_lib.ATTN_OK
+
+
+def test_w4a16_workspace_cache_is_zeroed_after_a_failed_status(monkeypatch):
+    """The split-K workspaces w4a16_matmul caches per (device, stream) hold tickets
+    that a timed-out launch may leave set: a device status other than ATTN_OK
+    zeroes every cached workspace; ATTN_OK leaves them alone. (Host logic only: a
+    fake library answers the status call and the cache holds CPU tensors.)"""
+    class FakeLib:
+        status = attn.ATTN_OK
+
+        def attn_get_device_status(self, stream):
+            return self.status
+
+    fake = FakeLib()
+    monkeypatch.setattr(attn, "load", lambda: fake)
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda *a, **k: None)
+    cache = {(0, 1): torch.full((64,), 7, dtype=torch.uint8), (0, 2): torch.full((32,), 9, dtype=torch.uint8)}
+    monkeypatch.setattr(attn, "_W4_WORKSPACES", cache)
+    assert attn.attn_get_device_status(None) == attn.ATTN_OK
+    assert all(bool((t != 0).all()) for t in cache.values())
+    fake.status = attn.ATTN_ERR_TIMEOUT
+    assert attn.attn_get_device_status(None) == attn.ATTN_ERR_TIMEOUT
+    assert all(int(t.count_nonzero()) == 0 for t in cache.values())
+    assert set(cache) == {(0, 1), (0, 2)}                  # kept, zeroed, not dropped
